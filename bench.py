@@ -1,0 +1,450 @@
+"""Benchmark of the exponent-split KV codec on B200.
+
+One step = the whole hot path over one batch: plan (histogram + codebook),
+encode and decode of every K and V tensor of the workload, one batched launch
+per kernel (default workload: Llama-3-8B KV after an 8192-token prefill, 32
+layers x {K, V} x [8192, 8, 128] bf16 = 1.07 GB).  Inputs are seeded synthetic
+tensors resident in HBM; the batch (1.07 GB) is larger than L2 (126 MB), so no
+flush is needed between steps.
+
+Prints one JSON line.  `value` is raw input bytes per second through a full
+round trip (plan + encode + decode); encode (plan + encode) and decode rates,
+per-kernel roofline fractions and the compression ratio ride along.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload llama3-8b|qwen3-32b-layer|...] [--mode batch|per_layer]
+
+`--impl reference` times the CPU oracle (plain single-threaded C) on a bounded
+sample of the same workload: the only reference implementation there is.
+For N > 1 (torchrun), every rank codes its own batch of the same size (weak
+scaling: the tensors are independent, no data-path collective); timing is the
+max over ranks.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import kvgen  # noqa: E402
+
+METRIC = "encode/decode GB/s (raw bytes) on 1 B200, % of HBM roofline, compression ratio"
+UNIT = "GB/s"
+
+
+# ------------------------------------------------------------ host logic
+
+def rank_layers(cfg_layers: int, rank: int, world: int):
+    """Layers coded by one rank: every rank gets a full batch of its own layers
+    (weak scaling).  Rank r uses layer indices r*L .. r*L + L - 1 of the seeded
+    generator, so ranks never code the same tensor."""
+    return list(range(rank * cfg_layers, (rank + 1) * cfg_layers))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+WORKLOADS = {
+    # name: (config, layers per step, description)
+    "llama3-8b": ("llama3-8b", None, "Llama-3-8B KV, 8192-token prefill: 32 layers x {K,V} x [8192,8,128] bf16"),
+    "qwen3-32b-layer": ("qwen3-32b", 1, "Qwen3-32B KV at 131072 tokens, one layer: {K,V} x [131072,8,128] bf16"),
+    "qwen3-30b-a3b-e5m2": ("qwen3-30b-a3b-e5m2", None, "Qwen3-30B-A3B KV, FP8 E5M2: 48 layers x {K,V} x [32768,4,128]"),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def gpu_uuid(device) -> str:
+    """nvidia-smi id of a torch device (its UUID, whatever CUDA_VISIBLE_DEVICES says)."""
+    u = str(torch.cuda.get_device_properties(device).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our arm
+
+class Workload:
+    def __init__(self, name: str, rank: int, world: int, device):
+        cfg_name, layers_per_step, desc = WORKLOADS[name]
+        self.name, self.desc = name, desc
+        self.cfg = kvgen.CONFIGS[cfg_name]
+        self.dtype = 1 if self.cfg.fp8 else 0
+        nl = self.cfg.layers if layers_per_step is None else layers_per_step
+        self.layers = rank_layers(nl, rank, world)
+        self.xs = [kvgen.kv_tensor(self.cfg, l % self.cfg.layers if world == 1 else l, kv, device=device)
+                   for l in self.layers for kv in (0, 1)]
+        self.n = [x.numel() for x in self.xs]
+        self.esize = 1 if self.cfg.fp8 else 2
+        self.raw_bytes = sum(self.n) * self.esize
+
+
+def run_ours(args, rank, world, device):
+    import fp8_kv_cache_exp_b200 as sz
+    wl = Workload(args.workload, rank, world, device)
+    dt = wl.dtype
+    T = len(wl.xs)
+    stream = torch.cuda.current_stream()
+    ws = sz.new_workspace(dt, wl.n)
+    plans = sz.new_plans(T)
+    caps = [sz.sz_max_compressed_size(dt, n) for n in wl.n]
+    outs = [torch.empty(c, dtype=torch.uint8, device=device) for c in caps]
+    decs = [torch.empty_like(x) for x in wl.xs]
+
+    if args.mode == "batch":
+        groups = [list(range(T))]
+    else:  # per layer: K and V of one layer per call
+        groups = [[2 * i, 2 * i + 1] for i in range(T // 2)]
+    ws_g = [sz.new_workspace(dt, [wl.n[i] for i in g]) for g in groups] if args.mode != "batch" else [ws]
+    plans_g = [plans[g[0]: g[-1] + 1] for g in groups]
+
+    def plan_all():
+        for g, w, p in zip(groups, ws_g, plans_g):
+            sz.sz_plan_batched(dt, [wl.xs[i] for i in g], w, p)
+
+    def encode_all():
+        for g, w, p in zip(groups, ws_g, plans_g):
+            sz.sz_encode_batched(dt, p, [wl.xs[i] for i in g], [outs[i] for i in g], w)
+
+    def decode_all():
+        for g, w in zip(groups, ws_g):
+            sz.sz_decode_batched(dt, [outs[i] for i in g], [decs[i] for i in g], w)
+
+    # correctness of this very configuration before timing
+    plan_all(); encode_all(); decode_all()
+    for w in ws_g:
+        st = sz.sz_last_device_status(w)
+        if st != 0:
+            raise RuntimeError("device status %s" % sz.sz_status_string(st))
+    for x, d in zip(wl.xs, decs):
+        if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
+            raise RuntimeError("round trip mismatch")
+    totals = sz.sz_compressed_sizes(plans)
+    stream_bytes = sum(totals)
+    E_total = 0
+    for i in range(T):
+        h = plans[i].cpu()
+        E_total += int(h[16:24].view(torch.int64).item())
+
+    for _ in range(args.warmup):
+        plan_all(); encode_all(); decode_all()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(gpu_uuid(device))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        plan_all()
+        ev[k][1].record(stream)
+        encode_all()
+        ev[k][2].record(stream)
+        decode_all()
+        ev[k][3].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    t_plan = sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K
+    t_enc = sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K
+    t_dec = sum(ev[k][2].elapsed_time(ev[k][3]) for k in range(K)) / K
+    for w in ws_g:
+        st = sz.sz_last_device_status(w)
+        if st != 0:
+            raise RuntimeError("device status after timing: %s" % sz.sz_status_string(st))
+
+    ms_step = max_over_ranks(total_ms / K, world, device)
+    raw_all = sum_over_ranks(float(wl.raw_bytes), world, device)
+    value = raw_all / (ms_step * 1e-3) / 1e9
+
+    peak, peak_kind = load_peaks()
+    launches_per_step = 3 * len(groups)
+    kern = {
+        "plan": {"ms": t_plan, "bytes": wl.raw_bytes + 64 * T},
+        "encode": {"ms": t_enc, "bytes": wl.raw_bytes + stream_bytes},
+        "decode": {"ms": t_dec, "bytes": stream_bytes + wl.raw_bytes},
+    }
+    for k in kern.values():
+        k["gbs"] = k["bytes"] / (k["ms"] * 1e-3) / 1e9
+        k["frac"] = k["gbs"] / peak
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(kern[dom]["gbs"], 1), "peak": peak,
+            "unit": "GB/s", "frac": round(kern[dom]["frac"], 4), "traffic": None,
+            "peak_source": peak_kind}
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8" if dt == 1 else "u16", "data": "synthetic (seeded generator, see DESIGN.md)",
+        "config": {"workload": wl.name, "desc": wl.desc, "tensors_per_rank": T,
+                   "raw_bytes_per_rank": wl.raw_bytes, "mode": "one batch" if args.mode == "batch" else "per layer",
+                   "l2": "inputs larger than L2 (%.2f GB per step per rank)" % (wl.raw_bytes / 1e9),
+                   "parallelism": "replicas" if world == 1 else "dp%d (independent tensors)" % world},
+        "encode_gbs": round(wl.raw_bytes / ((t_plan + t_enc) * 1e-3) / 1e9, 1),
+        "decode_gbs": round(wl.raw_bytes / (t_dec * 1e-3) / 1e9, 1),
+        "ratio": round(wl.raw_bytes / stream_bytes, 5),
+        "escape_fraction": round(E_total / sum(wl.n), 6),
+        "kernels": {k: {"ms": round(v["ms"], 4), "gbs": round(v["gbs"], 1), "frac": round(v["frac"], 4)}
+                    for k, v in kern.items()},
+        "roofline": roof,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    return res, wl
+
+
+def run_e2e(args, wl, device):
+    """Same metric through the C ABI with host buffers: pinned H2D of the raw batch,
+    plan + encode + decode, D2H of the decoded batch, all inside the timed region."""
+    import fp8_kv_cache_exp_b200 as sz
+    dt = wl.dtype
+    T = len(wl.xs)
+    host_in = [x.cpu().pin_memory() for x in wl.xs]
+    host_out = [torch.empty_like(h).pin_memory() for h in host_in]
+    dev_in = [torch.empty_like(x) for x in wl.xs]
+    dev_out = [torch.empty_like(x) for x in wl.xs]
+    ws = sz.new_workspace(dt, wl.n)
+    plans = sz.new_plans(T)
+    outs = [torch.empty(sz.sz_max_compressed_size(dt, n), dtype=torch.uint8, device=device) for n in wl.n]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        sz.sz_plan_batched(dt, dev_in, ws, plans)
+        sz.sz_encode_batched(dt, plans, dev_in, outs, ws)
+        sz.sz_decode_batched(dt, outs, dev_out, ws)
+        for d, h in zip(dev_out, host_out):
+            h.copy_(d, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    for h, g in zip(host_out, host_in):
+        if not torch.equal(h.view(torch.uint8), g.view(torch.uint8)):
+            raise RuntimeError("e2e round trip mismatch")
+    for _ in range(max(1, args.warmup // 2)):
+        step()
+    K = max(2, min(args.steps, 5))
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if sz.sz_last_device_status(ws) != 0:
+        raise RuntimeError("device status in e2e")
+    ms = a.elapsed_time(b) / K
+    return {"value": round(wl.raw_bytes / (ms * 1e-3) / 1e9, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": wl.raw_bytes, "d2h_bytes_per_step": wl.raw_bytes, "steps": K}
+
+
+# ------------------------------------------------------- the oracle arm
+
+def oracle_sample(cfg_name: str, budget_s: float):
+    """Time the CPU oracle (as it stands) on one layer's K and V: plan + encode + decode."""
+    import numpy as np
+    import oracle
+    cfg = kvgen.CONFIGS[cfg_name]
+    dt = 1 if cfg.fp8 else 0
+    xs = [kvgen.kv_tensor(cfg, 0, kv) for kv in (0, 1)]
+    raws = [x.contiguous().view(torch.uint8).reshape(-1).numpy() for x in xs]
+    nbytes = sum(r.size for r in raws)
+    t_enc = t_dec = 0.0
+    reps = 0
+    t_start = time.perf_counter()
+    while True:
+        for r in raws:
+            n = r.size // (2 if dt == 0 else 1)
+            t0 = time.perf_counter()
+            s = oracle.encode(dt, r)
+            t1 = time.perf_counter()
+            back = oracle.decode(s, n, dt)
+            t2 = time.perf_counter()
+            t_enc += t1 - t0
+            t_dec += t2 - t1
+            if not np.array_equal(back, r):
+                raise RuntimeError("oracle round trip mismatch")
+        reps += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    raw_total = nbytes * reps
+    return {
+        "value": round(raw_total / (t_enc + t_dec) / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "sample": "%s layer 0 K+V (%.1f MB raw) x %d rep(s), single-threaded C oracle" % (cfg_name, nbytes / 1e6, reps),
+        "encode_gbs": round(raw_total / t_enc / 1e9, 4), "decode_gbs": round(raw_total / t_dec / 1e9, 4),
+        "seconds": round(t_enc + t_dec, 2),
+    }
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg_name = WORKLOADS[args.workload][0]
+    sample = None
+    times = []
+    for k in range(args.warmup + args.steps):
+        r = oracle_sample(cfg_name, 0.0)
+        if k >= args.warmup:
+            times.append(r)
+        sample = r
+    val = statistics.median(t["value"] for t in times)
+    raw = 2 * kvgen.CONFIGS[cfg_name].numel * (1 if kvgen.CONFIGS[cfg_name].fp8 else 2)
+    ms = raw / (val * 1e9) * 1e3
+    cpu = dict(sample)
+    cpu["value"] = val
+    return {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8" if kvgen.CONFIGS[cfg_name].fp8 else "u16", "data": "synthetic",
+        "config": {"workload": args.workload, "desc": WORKLOADS[args.workload][2],
+                   "sample": cpu["sample"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3-8b")
+    ap.add_argument("--mode", choices=["batch", "per_layer"], default="batch")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        res, wl = run_ours(args, rank, world, device)
+        if not args.no_e2e:
+            e2e = run_e2e(args, wl, device)
+            e2e_val = sum_over_ranks(wl.raw_bytes, world, device) / (
+                max_over_ranks(e2e["ms_per_step"], world, device) * 1e-3) / 1e9
+            e2e["value"] = round(e2e_val, 2)
+            res["e2e"] = e2e
+        if rank == 0 and world == 1 and args.cpu_baseline_seconds > 0:
+            res["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload][0], args.cpu_baseline_seconds)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+"""Python binding of libsplitzip: lossless exponent-split coding of BF16 / FP8 E5M2
+KV-cache tensors on a B200 GPU (SplitZip project page, Abstract and FAQ).
+
+Argument marshalling only: the functions below have the names of the C ABI in
+include/splitzip.h and pass torch tensors' device pointers and the current CUDA
+stream to it.  Every step of the codec runs in the library's CUDA kernels.
+Importing this package loads libsplitzip.so and raises ImportError if it has not
+been built (python -m fp8_kv_cache_exp_b200.build); there is no other path.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SZ_BF16", "SZ_FP8_E5M2", "SZ_OK", "SplitZipError", "lib", "lib_path",
+    "sz_status_string", "sz_workspace_bytes", "sz_workspace_bytes_batched", "sz_stream_bytes",
+    "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
+    "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched", "sz_decode",
+    "sz_decode_batched", "sz_last_device_status", "dtype_of", "elem_bytes", "numel_of",
+    "new_workspace", "new_plans",
+]
+
+SZ_BF16 = 0
+SZ_FP8_E5M2 = 1
+
+SZ_OK = 0
+SZ_ERR_INVALID_ARG = 1
+SZ_ERR_UNSUPPORTED_DTYPE = 2
+SZ_ERR_BUFFER_TOO_SMALL = 3
+SZ_ERR_CORRUPT_STREAM = 4
+SZ_ERR_CUDA = 5
+SZ_ERR_TIMEOUT = 6
+SZ_ERR_PLAN_MISMATCH = 7
+SZ_ERR_INTERNAL = 8
+
+SZ_HEADER_BYTES = 64
+SZ_BLOCK_ELEMS = 4096
+SZ_MAX_BATCH = 256
+
+lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitzip.so")
+
+
+def _load():
+    if not os.path.exists(lib_path):
+        raise ImportError("libsplitzip.so is not built (%s); run: python -m fp8_kv_cache_exp_b200.build"
+                          % lib_path)
+    L = ctypes.CDLL(lib_path)
+    vp, u64, sz, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_int
+    pvp, pu64, psz = ctypes.POINTER(vp), ctypes.POINTER(u64), ctypes.POINTER(sz)
+    sigs = {
+        "sz_status_string": (ctypes.c_char_p, [i32]),
+        "sz_workspace_bytes": (sz, [i32, u64]),
+        "sz_workspace_bytes_batched": (sz, [i32, i32, pu64]),
+        "sz_stream_bytes": (sz, [i32, u64, u64]),
+        "sz_max_compressed_size": (sz, [i32, u64]),
+        "sz_workspace_init": (i32, [vp, sz, vp]),
+        "sz_plan": (i32, [i32, vp, u64, vp, sz, vp, vp]),
+        "sz_plan_batched": (i32, [i32, i32, pvp, pu64, vp, sz, vp, vp]),
+        "sz_compressed_size": (i32, [vp, pu64, vp]),
+        "sz_compressed_sizes": (i32, [i32, vp, pu64, vp]),
+        "sz_encode": (i32, [i32, vp, vp, u64, vp, sz, vp, sz, vp]),
+        "sz_encode_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, sz, vp]),
+        "sz_decode": (i32, [i32, vp, sz, vp, u64, vp, sz, vp]),
+        "sz_decode_batched": (i32, [i32, i32, pvp, psz, pvp, pu64, vp, sz, vp]),
+        "sz_last_device_status": (i32, [vp, vp]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+class SplitZipError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        super().__init__("%s%s (status %d)" % (where + ": " if where else "",
+                                              sz_status_string(status), self.status))
+
+
+def sz_status_string(status: int) -> str:
+    return lib.sz_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != SZ_OK:
+        raise SplitZipError(status, where)
+
+
+def dtype_of(x: torch.Tensor) -> int:
+    """Codec dtype of a tensor: bfloat16 -> SZ_BF16, float8_e5m2 -> SZ_FP8_E5M2."""
+    if x.dtype == torch.bfloat16:
+        return SZ_BF16
+    if x.dtype == torch.float8_e5m2:
+        return SZ_FP8_E5M2
+    raise TypeError("unsupported tensor dtype %s (bfloat16 or float8_e5m2)" % x.dtype)
+
+
+def elem_bytes(dtype: int) -> int:
+    return 2 if dtype == SZ_BF16 else 1
+
+
+def numel_of(x: torch.Tensor, dtype: int) -> int:
+    """Elements of the codec dtype held by a tensor (any torch dtype view)."""
+    return x.numel() * x.element_size() // elem_bytes(dtype)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _p(x: torch.Tensor):
+    return ctypes.c_void_p(x.data_ptr())
+
+
+def _arr(ctype, values):
+    values = list(values)
+    return (ctype * len(values))(*values)
+
+
+# ------------------------------------------------------------------- sizes
+
+def sz_workspace_bytes(dtype: int, n: int) -> int:
+    return int(lib.sz_workspace_bytes(dtype, n))
+
+
+def sz_workspace_bytes_batched(dtype: int, ns) -> int:
+    ns = list(ns)
+    return int(lib.sz_workspace_bytes_batched(dtype, len(ns), _arr(ctypes.c_uint64, ns)))
+
+
+def sz_stream_bytes(dtype: int, n: int, E: int) -> int:
+    return int(lib.sz_stream_bytes(dtype, n, E))
+
+
+def sz_max_compressed_size(dtype: int, n: int) -> int:
+    return int(lib.sz_max_compressed_size(dtype, n))
+
+
+def new_workspace(dtype: int, ns, device="cuda", stream=None) -> torch.Tensor:
+    """A zero-initialised workspace for a batch with element counts ns."""
+    ws = torch.empty(sz_workspace_bytes_batched(dtype, ns), dtype=torch.uint8, device=device)
+    sz_workspace_init(ws, stream)
+    return ws
+
+
+def new_plans(T: int, device="cuda") -> torch.Tensor:
+    return torch.zeros((T, SZ_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------- the calls
+
+def sz_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib.sz_workspace_init(_p(ws), ws.nbytes, _stream(stream)), "sz_workspace_init")
+
+
+def sz_plan(dtype: int, x: torch.Tensor, ws: torch.Tensor, plan: torch.Tensor, stream=None):
+    _check(lib.sz_plan(dtype, _p(x), numel_of(x, dtype), _p(ws), ws.nbytes, _p(plan),
+                       _stream(stream)), "sz_plan")
+
+
+def sz_plan_batched(dtype: int, xs, ws: torch.Tensor, plans: torch.Tensor, stream=None):
+    xs = list(xs)
+    T = len(xs)
+    _check(lib.sz_plan_batched(dtype, T, _arr(ctypes.c_void_p, [x.data_ptr() for x in xs]),
+                               _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs]),
+                               _p(ws), ws.nbytes, _p(plans), _stream(stream)), "sz_plan_batched")
+
+
+def sz_compressed_size(plan: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_uint64(0)
+    _check(lib.sz_compressed_size(_p(plan), ctypes.byref(out), _stream(stream)), "sz_compressed_size")
+    return int(out.value)
+
+
+def sz_compressed_sizes(plans: torch.Tensor, stream=None):
+    T = plans.shape[0]
+    out = (ctypes.c_uint64 * T)()
+    _check(lib.sz_compressed_sizes(T, _p(plans), out, _stream(stream)), "sz_compressed_sizes")
+    return [int(v) for v in out]
+
+
+def sz_encode(dtype: int, plan: torch.Tensor, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+              stream=None):
+    _check(lib.sz_encode(dtype, _p(plan), _p(x), numel_of(x, dtype), _p(out), out.nbytes, _p(ws),
+                         ws.nbytes, _stream(stream)), "sz_encode")
+
+
+def sz_encode_batched(dtype: int, plans: torch.Tensor, xs, outs, ws: torch.Tensor, stream=None):
+    xs, outs = list(xs), list(outs)
+    T = len(xs)
+    _check(lib.sz_encode_batched(
+        dtype, T, _p(plans), _arr(ctypes.c_void_p, [x.data_ptr() for x in xs]),
+        _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs]),
+        _arr(ctypes.c_void_p, [o.data_ptr() for o in outs]),
+        _arr(ctypes.c_size_t, [o.nbytes for o in outs]), _p(ws), ws.nbytes, _stream(stream)),
+        "sz_encode_batched")
+
+
+def sz_decode(dtype: int, comp: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, comp_bytes=None,
+              stream=None):
+    cb = comp.nbytes if comp_bytes is None else int(comp_bytes)
+    _check(lib.sz_decode(dtype, _p(comp), cb, _p(out), numel_of(out, dtype), _p(ws), ws.nbytes,
+                         _stream(stream)), "sz_decode")
+
+
+def sz_decode_batched(dtype: int, comps, outs, ws: torch.Tensor, comp_bytes=None, stream=None):
+    comps, outs = list(comps), list(outs)
+    T = len(comps)
+    cbs = [c.nbytes for c in comps] if comp_bytes is None else [int(b) for b in comp_bytes]
+    _check(lib.sz_decode_batched(
+        dtype, T, _arr(ctypes.c_void_p, [c.data_ptr() for c in comps]), _arr(ctypes.c_size_t, cbs),
+        _arr(ctypes.c_void_p, [o.data_ptr() for o in outs]),
+        _arr(ctypes.c_uint64, [numel_of(o, dtype) for o in outs]), _p(ws), ws.nbytes,
+        _stream(stream)), "sz_decode_batched")
+
+
+def sz_last_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise; return (and clear) the workspace's device error word."""
+    return int(lib.sz_last_device_status(_p(ws), _stream(stream)))

@@ -1,0 +1,208 @@
+// sz_api.cu -- the extern "C" entry points of libsplitzip (see include/splitzip.h).
+// Host-side argument checks, workspace partitioning and kernel dispatch.  No
+// device memory is allocated here; every device buffer belongs to the caller.
+#include <cuda_runtime.h>
+
+#include "splitzip.h"
+#include "sz_common.cuh"
+#include "sz_internal.h"
+
+namespace {
+
+using namespace sz;
+
+bool dtype_ok(sz_dtype d) { return d == SZ_BF16 || d == SZ_FP8_E5M2; }
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+uint64_t total_tiles(int T, const uint64_t *n) {
+    uint64_t s = 0;
+    for (int t = 0; t < T; ++t) s += cdiv(n[t], kBlock);
+    return s;
+}
+
+int num_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+// Shared checks of a batch: dtype, T, element counts, workspace.
+sz_status check_batch(sz_dtype dtype, int T, const uint64_t *n, const void *d_ws, size_t ws_bytes) {
+    if (!dtype_ok(dtype)) return SZ_ERR_UNSUPPORTED_DTYPE;
+    if (T < 1 || T > SZ_MAX_BATCH || !n || !d_ws || !aligned(d_ws, 8)) return SZ_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t)
+        if (n[t] >= (1ull << 32)) return SZ_ERR_INVALID_ARG;
+    if (ws_bytes < sz_workspace_bytes_batched(dtype, T, n)) return SZ_ERR_BUFFER_TOO_SMALL;
+    return SZ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sz_status_string(sz_status s) {
+    switch (s) {
+        case SZ_OK: return "ok";
+        case SZ_ERR_INVALID_ARG: return "invalid argument";
+        case SZ_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+        case SZ_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+        case SZ_ERR_CORRUPT_STREAM: return "corrupt stream";
+        case SZ_ERR_CUDA: return "CUDA runtime error";
+        case SZ_ERR_TIMEOUT: return "look-back wait timed out";
+        case SZ_ERR_PLAN_MISMATCH: return "data or sizes do not match the plan";
+        case SZ_ERR_INTERNAL: return "internal consistency check failed";
+    }
+    return "unknown status";
+}
+
+size_t sz_workspace_bytes_batched(sz_dtype dtype, int T, const uint64_t *n) {
+    if (!dtype_ok(dtype) || T < 1 || T > SZ_MAX_BATCH || !n) return 0;
+    return ws_layout(T, total_tiles(T, n)).bytes;
+}
+
+size_t sz_workspace_bytes(sz_dtype dtype, uint64_t n) { return sz_workspace_bytes_batched(dtype, 1, &n); }
+
+size_t sz_stream_bytes(sz_dtype dtype, uint64_t n, uint64_t E) {
+    if (!dtype_ok(dtype)) return 0;
+    return stream_layout(dtype, n, E).total;
+}
+
+size_t sz_max_compressed_size(sz_dtype dtype, uint64_t n) { return sz_stream_bytes(dtype, n, n); }
+
+sz_status sz_workspace_init(void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!d_ws || !aligned(d_ws, 8) || ws_bytes < size_t(kCtlWords) * 4) return SZ_ERR_INVALID_ARG;
+    return cudaMemsetAsync(d_ws, 0, ws_bytes, stream) == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+}
+
+sz_status sz_plan_batched(sz_dtype dtype, int T, const void *const *d_in, const uint64_t *n,
+                          void *d_ws, size_t ws_bytes, sz_plan_t *d_plans, cudaStream_t stream) {
+    sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
+    if (s != SZ_OK) return s;
+    if (!d_in || !d_plans || !aligned(d_plans, 8)) return SZ_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t)
+        if (n[t] && (!d_in[t] || !aligned(d_in[t], 16))) return SZ_ERR_INVALID_ARG;
+    const WsLayout w = ws_layout(T, total_tiles(T, n));
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    PlanArgs a;
+    a.dtype = dtype;
+    a.T = T;
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return SZ_ERR_CUDA;
+    a.in = d_in;
+    a.n = n;
+    a.ctl = reinterpret_cast<uint32_t *>(ws);
+    a.hist = reinterpret_cast<uint32_t *>(ws + w.hist);
+    a.ticket = reinterpret_cast<uint32_t *>(ws + w.ticket);
+    a.plans = reinterpret_cast<uint8_t *>(d_plans);
+    return launch_plan(a, stream);
+}
+
+sz_status sz_plan(sz_dtype dtype, const void *d_in, uint64_t n, void *d_ws, size_t ws_bytes,
+                  sz_plan_t *d_plan, cudaStream_t stream) {
+    const void *in[1] = {d_in};
+    return sz_plan_batched(dtype, 1, in, &n, d_ws, ws_bytes, d_plan, stream);
+}
+
+sz_status sz_compressed_sizes(int T, const sz_plan_t *d_plans, uint64_t *h_bytes,
+                              cudaStream_t stream) {
+    if (T < 1 || T > SZ_MAX_BATCH || !d_plans || !h_bytes) return SZ_ERR_INVALID_ARG;
+    sz_plan_t host[SZ_MAX_BATCH];
+    if (cudaMemcpyAsync(host, d_plans, sizeof(sz_plan_t) * T, cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return SZ_ERR_CUDA;
+    for (int t = 0; t < T; ++t) {
+        uint64_t v = 0;
+        for (int b = 0; b < 8; ++b) v |= uint64_t(host[t].bytes[40 + b]) << (8 * b);
+        h_bytes[t] = v;
+    }
+    return SZ_OK;
+}
+
+sz_status sz_compressed_size(const sz_plan_t *d_plan, uint64_t *h_bytes, cudaStream_t stream) {
+    return sz_compressed_sizes(1, d_plan, h_bytes, stream);
+}
+
+sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
+                            const void *const *d_in, const uint64_t *n, void *const *d_out,
+                            const size_t *out_cap, void *d_ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+    sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
+    if (s != SZ_OK) return s;
+    if (!d_plans || !aligned(d_plans, 8) || !d_in || !d_out || !out_cap) return SZ_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        if (n[t] && (!d_in[t] || !aligned(d_in[t], 16))) return SZ_ERR_INVALID_ARG;
+        if (!d_out[t] || !aligned(d_out[t], 16)) return SZ_ERR_INVALID_ARG;
+        // the smallest stream for n (no escapes) must fit in any case
+        if (out_cap[t] < stream_layout(dtype, n[t], 0).total) return SZ_ERR_BUFFER_TOO_SMALL;
+    }
+    const uint64_t tiles = total_tiles(T, n);
+    const WsLayout w = ws_layout(T, tiles);
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    EncodeArgs a;
+    a.dtype = dtype;
+    a.T = T;
+    a.num_sms = num_sms();
+    a.plans = reinterpret_cast<const uint8_t *>(d_plans);
+    a.in = d_in;
+    a.n = n;
+    a.out = d_out;
+    a.cap = out_cap;
+    a.ctl = reinterpret_cast<uint32_t *>(ws);
+    a.status = reinterpret_cast<unsigned long long *>(ws + w.status);
+    return launch_encode(a, stream);
+}
+
+sz_status sz_encode(sz_dtype dtype, const sz_plan_t *d_plan, const void *d_in, uint64_t n,
+                    void *d_out, size_t out_cap, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    const void *in[1] = {d_in};
+    void *out[1] = {d_out};
+    return sz_encode_batched(dtype, 1, d_plan, in, &n, out, &out_cap, d_ws, ws_bytes, stream);
+}
+
+sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,
+                            const size_t *comp_bytes, void *const *d_out, const uint64_t *n,
+                            void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
+    if (s != SZ_OK) return s;
+    if (!d_comp || !comp_bytes || !d_out) return SZ_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        if (!d_comp[t] || !aligned(d_comp[t], 16)) return SZ_ERR_INVALID_ARG;
+        if (n[t] && (!d_out[t] || !aligned(d_out[t], 16))) return SZ_ERR_INVALID_ARG;
+        // every plane of an n-element stream must lie inside the buffer
+        if (comp_bytes[t] < stream_layout(dtype, n[t], 0).total) return SZ_ERR_CORRUPT_STREAM;
+    }
+    DecodeArgs a;
+    a.dtype = dtype;
+    a.T = T;
+    a.num_sms = num_sms();
+    a.comp = d_comp;
+    a.comp_bytes = comp_bytes;
+    a.out = d_out;
+    a.n = n;
+    a.ctl = static_cast<uint32_t *>(d_ws);
+    return launch_decode(a, stream);
+}
+
+sz_status sz_decode(sz_dtype dtype, const void *d_comp, size_t comp_bytes, void *d_out, uint64_t n,
+                    void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    const void *comp[1] = {d_comp};
+    void *out[1] = {d_out};
+    return sz_decode_batched(dtype, 1, comp, &comp_bytes, out, &n, d_ws, ws_bytes, stream);
+}
+
+sz_status sz_last_device_status(void *d_ws, cudaStream_t stream) {
+    if (!d_ws || !aligned(d_ws, 8)) return SZ_ERR_INVALID_ARG;
+    uint32_t err[2] = {0, 0};
+    if (cudaMemcpyAsync(err, d_ws, sizeof(err), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return SZ_ERR_CUDA;
+    if (err[0] != 0) {
+        if (cudaMemsetAsync(d_ws, 0, sizeof(err), stream) != cudaSuccess) return SZ_ERR_CUDA;
+    }
+    return static_cast<sz_status>(err[0]);
+}
+
+}  // extern "C"

@@ -1,0 +1,253 @@
+// sz_common.cuh -- definitions shared by the libsplitzip kernels and host layer:
+// stream-format layout (format v1), workspace layout, launch parameter blocks
+// and small device helpers.
+//
+// Method: "SplitZip: Ultra-Fast Lossless KV Compression for Disaggregated LLM
+// Serving" (project page), Abstract: frequent exponents -> fixed 4-bit codes,
+// sign and mantissa exact, rare exponents -> sparse escape stream.  The byte
+// layout is this library's own (the page prints none); it is described in
+// include/splitzip.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "splitzip.h"
+
+namespace sz {
+
+constexpr uint32_t kMagic = 0x564B5A53u;  // "SZKV" little-endian
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kBlockLog2 = 12;
+constexpr uint32_t kBlock = 1u << kBlockLog2;  // elements per escape-offset block (= one tile)
+constexpr uint32_t kCodes = 15;                // codes 0..14 name codebook entries
+constexpr uint32_t kEscape = 15;               // code 15 marks an escaped exponent
+constexpr int kTileThreads = 256;              // threads per encode/decode tile CTA
+constexpr int kSmallBatch = 8;                 // parameter blocks sized for <= 8 tensors ...
+constexpr int kLargeBatch = SZ_MAX_BATCH;      // ... or for up to SZ_MAX_BATCH tensors
+
+// Control words at the start of every workspace (u32 each).
+enum : int {
+    kCtlErr = 0,       // first device error (sz_status), 0 if none
+    kCtlErrDetail = 1, // error detail (e.g. the tile that failed)
+    kCtlEpoch = 2,     // encode launch counter, tags look-back status words
+    kCtlTileCtr = 3,   // encode job counter (tile ids in launch order)
+    kCtlDone = 4,      // encode CTAs finished
+    kCtlWords = 64     // 256 bytes reserved
+};
+
+__host__ __device__ constexpr uint64_t align256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
+__host__ __device__ constexpr uint64_t cdiv(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+
+template <int DT> struct Dt;
+template <> struct Dt<SZ_BF16> {
+    static constexpr int kBins = 256;      // 8-bit exponent
+    static constexpr int kElemBytes = 2;
+};
+template <> struct Dt<SZ_FP8_E5M2> {
+    static constexpr int kBins = 32;       // 5-bit exponent
+    static constexpr int kElemBytes = 1;
+};
+
+// Section offsets of a stream with n elements and E escapes.
+struct Layout {
+    uint64_t nb;         // 4096-element blocks
+    uint64_t tab_end;    // end of the offsets table: 64 + 4(nb+1)
+    uint64_t plane[3];   // BF16: sm, code ; E5M2: sign, mantissa, code
+    uint64_t plane_len[3];
+    int nplanes;
+    uint64_t code;       // code-plane start (the last plane)
+    uint64_t esc;        // escape-stream start
+    uint64_t total;      // stream length
+};
+
+__host__ __device__ inline Layout stream_layout(int dtype, uint64_t n, uint64_t E) {
+    Layout L;
+    L.nb = cdiv(n, kBlock);
+    L.tab_end = 64 + 4 * (L.nb + 1);
+    if (dtype == SZ_BF16) {
+        L.nplanes = 2;
+        L.plane_len[0] = n;
+        L.plane_len[1] = cdiv(n, 2);
+        L.plane_len[2] = 0;
+    } else {
+        L.nplanes = 3;
+        L.plane_len[0] = cdiv(n, 8);
+        L.plane_len[1] = cdiv(n, 4);
+        L.plane_len[2] = cdiv(n, 2);
+    }
+    uint64_t pos = align256(L.tab_end);
+#if defined(__CUDA_ARCH__)
+#pragma unroll
+#endif
+    for (int s = 0; s < 3; ++s) {
+        L.plane[s] = pos;
+        if (s < L.nplanes) pos = align256(pos + L.plane_len[s]);
+    }
+    L.code = L.plane[L.nplanes - 1];
+    L.esc = pos;
+    L.total = pos + E;
+    return L;
+}
+
+// Workspace partition: control block, per-tensor histograms and tickets
+// (plan), per-tile look-back status words (encode).
+struct WsLayout {
+    size_t hist, ticket, status, bytes;
+};
+inline WsLayout ws_layout(int T, uint64_t total_tiles) {
+    WsLayout w;
+    w.hist = kCtlWords * 4;
+    w.ticket = w.hist + size_t(T) * 256 * 4;
+    w.status = w.ticket + align256(size_t(T) * 4);
+    w.bytes = w.status + size_t(total_tiles) * 8;
+    return w;
+}
+
+// ------------------------------------------------------------- parameters
+// Passed by value as __grid_constant__ kernel parameters: no descriptor copy.
+
+template <int MAXB>
+struct PlanParams {
+    uint32_t *ctl;
+    uint32_t *hist;      // T x 256 counts
+    uint32_t *ticket;    // T items-done counters
+    uint8_t *plans;      // T x 64-byte plans
+    uint64_t total_items;
+    int T;
+    const uint8_t *in[MAXB];
+    uint64_t n[MAXB];
+    uint64_t item_begin[MAXB + 1];  // prefix over tensors of ceil(n / item elements)
+};
+
+template <int MAXB>
+struct EncodeParams {
+    uint32_t *ctl;
+    unsigned long long *status;  // one look-back word per global tile
+    const uint8_t *plans;
+    uint32_t total_tiles;
+    uint32_t total_jobs;         // tiles + empty tensors
+    int T;
+    int n_empty;
+    const uint8_t *in[MAXB];
+    uint8_t *out[MAXB];
+    uint64_t n[MAXB];
+    uint64_t cap[MAXB];
+    uint32_t tile_begin[MAXB + 1];
+    uint16_t empty[MAXB];
+};
+
+template <int MAXB>
+struct DecodeParams {
+    uint32_t *ctl;
+    uint32_t total_tiles;
+    int T;
+    const uint8_t *comp[MAXB];
+    uint64_t comp_bytes[MAXB];
+    uint8_t *out[MAXB];
+    uint64_t n[MAXB];
+    uint32_t tile_begin[MAXB + 1];
+};
+
+// ---------------------------------------------------------- device helpers
+
+// Record the first device error; later errors keep the first one.
+__device__ inline void set_error(uint32_t *ctl, uint32_t code, uint32_t detail) {
+    if (atomicCAS(&ctl[kCtlErr], 0u, code) == 0u) atomicExch(&ctl[kCtlErrDetail], detail);
+}
+
+__device__ inline uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ inline unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ inline void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ inline uint32_t ld_relaxed_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Index t with begin[t] <= x < begin[t+1] (begin non-decreasing, begin[0] = 0).
+template <typename U, int MAXB>
+__device__ inline int find_tensor(const U (&begin)[MAXB + 1], int T, U x) {
+    int lo = 0, hi = T;  // invariant: begin[lo] <= x < begin[hi]
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (begin[mid] <= x) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Exclusive prefix sum over the CTA (NT threads); *total receives the sum.
+template <int NT>
+__device__ inline uint32_t block_exclusive_scan(uint32_t v, uint32_t *s_warp, uint32_t *total) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    uint32_t before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        uint32_t s = s_warp[w];
+        before += (w < warp) ? s : 0u;
+        all += s;
+    }
+    *total = all;
+    return before + x - v;
+}
+
+// w[i] for a small runtime index without spilling the array to local memory.
+__device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t i) {
+    const uint32_t lo = (i & 1u) ? w1 : w0;
+    const uint32_t hi = (i & 1u) ? w3 : w2;
+    return (i & 2u) ? hi : lo;
+}
+
+// Plan words (the 64-byte header as 16 little-endian u32 words).
+struct Header {
+    uint32_t magic, vtag;  // vtag = version | dtype << 16 | block_log2 << 24
+    uint64_t n, E, total;
+    uint32_t cbw[4];       // cb[0..14] in bytes 0..14, byte 15 zero
+};
+
+__device__ inline Header load_header(const uint8_t *h) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(h);
+    Header H;
+    H.magic = w[0];
+    H.vtag = w[1];
+    H.n = uint64_t(w[2]) | (uint64_t(w[3]) << 32);
+    H.E = uint64_t(w[4]) | (uint64_t(w[5]) << 32);
+    H.cbw[0] = w[6];
+    H.cbw[1] = w[7];
+    H.cbw[2] = w[8];
+    H.cbw[3] = w[9];
+    H.total = uint64_t(w[10]) | (uint64_t(w[11]) << 32);
+    return H;
+}
+
+__device__ inline uint32_t header_vtag(int dtype) {
+    return kVersion | (uint32_t(dtype) << 16) | (kBlockLog2 << 24);
+}
+
+__device__ inline uint32_t cb_byte(const uint32_t (&cbw)[4], int c) {
+    return (pick4(cbw[0], cbw[1], cbw[2], cbw[3], uint32_t(c) >> 2) >> (8 * (c & 3))) & 0xFFu;
+}
+
+}  // namespace sz

@@ -1,0 +1,44 @@
+// sz_internal.h -- launcher interface between the C ABI layer and the kernels.
+// Host arrays are read during the call only (copied into kernel parameters).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "splitzip.h"
+
+namespace sz {
+
+struct PlanArgs {
+    int dtype, T, num_sms;
+    const void *const *in;
+    const uint64_t *n;
+    uint32_t *ctl, *hist, *ticket;
+    uint8_t *plans;
+};
+
+struct EncodeArgs {
+    int dtype, T, num_sms;
+    const uint8_t *plans;
+    const void *const *in;
+    const uint64_t *n;
+    void *const *out;
+    const size_t *cap;
+    uint32_t *ctl;
+    unsigned long long *status;
+};
+
+struct DecodeArgs {
+    int dtype, T, num_sms;
+    const void *const *comp;
+    const size_t *comp_bytes;
+    void *const *out;
+    const uint64_t *n;
+    uint32_t *ctl;
+};
+
+sz_status launch_plan(const PlanArgs &a, cudaStream_t stream);
+sz_status launch_encode(const EncodeArgs &a, cudaStream_t stream);
+sz_status launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+}  // namespace sz

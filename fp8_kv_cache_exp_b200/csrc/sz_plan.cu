@@ -1,0 +1,303 @@
+// sz_plan.cu -- plan kernel: exponent histogram + top-15 codebook selection.
+//
+// SplitZip project page, Abstract: the codec gives fixed 4-bit codes to "the
+// most frequent exponent values".  This kernel counts every exponent value of
+// each tensor and, in the last CTA to finish a tensor, ranks the values by
+// (count descending, value ascending), takes the first 15 as the codebook and
+// writes the 64-byte plan (= stream header: n, E, codebook, total bytes).
+//
+// Histogram design (B200): each thread owns a private column of packed 16-bit
+// counters in shared memory (word r of thread t at s_cols[r * NT + t] holds
+// the counts of exponent values 2r and 2r+1).  Lane t of every warp always
+// touches bank t % 32, so the shared-memory atomics never conflict and never
+// contend, whatever the exponent distribution (an all-zero tensor costs the
+// same as a spread one).  Counters are flushed to the tensor's global
+// histogram (one atomic per non-zero bin per CTA) before any thread can have
+// counted 65535 elements.  Input is streamed with 16-byte read-only loads, a
+// software-pipelined batch of U vectors per thread in flight.
+#include "sz_common.cuh"
+#include "sz_internal.h"
+
+namespace sz {
+
+namespace {
+
+constexpr int kPlanThreads = 256;
+constexpr int kPlanUnroll = 8;                // 16-byte vectors in flight per thread
+constexpr uint32_t kItemBytes = 16384;        // partition unit of the input
+constexpr uint32_t kMaxPerThread = 65535;     // 16-bit counter limit
+
+template <int DT>
+struct PlanCfg {
+    static constexpr int kBins = Dt<DT>::kBins;
+    static constexpr int kRows = kBins / 2;                 // packed counter words per thread
+    static constexpr int kElemBytes = Dt<DT>::kElemBytes;
+    static constexpr int kVecElems = 16 / kElemBytes;       // elements per 16-byte vector
+    static constexpr uint32_t kItemElems = kItemBytes / kElemBytes;
+};
+
+// Count the elements of one 16-byte vector into this thread's column.
+template <int DT, int NT>
+__device__ __forceinline__ void count_vec(uint32_t *col, uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if constexpr (DT == SZ_BF16) {
+            // two elements per word: exponent bits 7..14 and 23..30
+            const uint32_t e0 = (w[k] >> 7) & 0xFFu, e1 = (w[k] >> 23) & 0xFFu;
+            atomicAdd(col + (e0 >> 1) * NT, 1u << ((e0 & 1u) << 4));
+            atomicAdd(col + (e1 >> 1) * NT, 1u << ((e1 & 1u) << 4));
+        } else {
+            // four elements per word: exponent bits 2..6 of each byte
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t e = (w[k] >> (8 * b + 2)) & 0x1Fu;
+                atomicAdd(col + (e >> 1) * NT, 1u << ((e & 1u) << 4));
+            }
+        }
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t exponent_scalar(const uint8_t *in, uint64_t i) {
+    if constexpr (DT == SZ_BF16) {
+        const uint32_t b = reinterpret_cast<const uint16_t *>(in)[i];
+        return (b >> 7) & 0xFFu;
+    } else {
+        return (uint32_t(in[i]) >> 2) & 0x1Fu;
+    }
+}
+
+// Count elements [a, b) of one tensor (a is a multiple of the vector size).
+template <int DT, int NT>
+__device__ void count_range(uint32_t *col, const uint8_t *in, uint64_t a, uint64_t b) {
+    using C = PlanCfg<DT>;
+    constexpr int U = kPlanUnroll;
+    const uint4 *src = reinterpret_cast<const uint4 *>(in) + a / C::kVecElems;
+    const uint64_t nvec = (b - a) / C::kVecElems;
+    const int tid = threadIdx.x;
+    uint4 cur[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const uint64_t k = uint64_t(tid) + uint64_t(u) * NT;
+        cur[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+    }
+    for (uint64_t base = 0; base < nvec; base += uint64_t(U) * NT) {
+        uint4 nxt[U];
+        const uint64_t nbase = base + uint64_t(U) * NT;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint64_t k = nbase + tid + uint64_t(u) * NT;
+            nxt[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint64_t k = base + tid + uint64_t(u) * NT;
+            if (k < nvec) count_vec<DT, NT>(col, cur[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+    }
+    // ragged end (< one vector): thread 0 counts it element by element
+    if (tid == 0) {
+        for (uint64_t i = a + nvec * C::kVecElems; i < b; ++i) {
+            const uint32_t e = exponent_scalar<DT>(in, i);
+            atomicAdd(col + (e >> 1) * NT, 1u << ((e & 1u) << 4));
+        }
+    }
+}
+
+// Add every thread's column into the global histogram g_hist and clear them.
+template <int DT, int NT>
+__device__ void flush_columns(uint32_t *s_cols, uint32_t *g_hist) {
+    using C = PlanCfg<DT>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    for (int r = warp; r < C::kRows; r += NT / 32) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int c = lane; c < NT; c += 32) {
+            const uint32_t w = s_cols[r * NT + c];
+            s_cols[r * NT + c] = 0;
+            lo += w & 0xFFFFu;
+            hi += w >> 16;
+        }
+        lo = __reduce_add_sync(0xffffffffu, lo);
+        hi = __reduce_add_sync(0xffffffffu, hi);
+        if (lane == 0) {
+            if (lo) atomicAdd(g_hist + 2 * r, lo);
+            if (hi) atomicAdd(g_hist + 2 * r + 1, hi);
+        }
+    }
+    __threadfence();
+    __syncthreads();
+}
+
+// Write a 64-byte plan (16 words) from thread-0 values kept in shared memory.
+__device__ inline void store_plan(uint8_t *plan, const uint32_t *s_words) {
+    if (threadIdx.x < 16) reinterpret_cast<uint32_t *>(plan)[threadIdx.x] = s_words[threadIdx.x];
+}
+
+__device__ inline void make_plan_words(uint32_t *s_words, int dtype, uint64_t n, uint64_t E,
+                                       const uint8_t *cb) {
+    const Layout L = stream_layout(dtype, n, E);
+    s_words[0] = kMagic;
+    s_words[1] = header_vtag(dtype);
+    s_words[2] = uint32_t(n);
+    s_words[3] = uint32_t(n >> 32);
+    s_words[4] = uint32_t(E);
+    s_words[5] = uint32_t(E >> 32);
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w = 0;
+        for (int b = 0; b < 4; ++b) {
+            const int c = 4 * q + b;
+            if (c < int(kCodes)) w |= uint32_t(cb[c]) << (8 * b);
+        }
+        s_words[6 + q] = w;
+    }
+    s_words[10] = uint32_t(L.total);
+    s_words[11] = uint32_t(L.total >> 32);
+    s_words[12] = s_words[13] = s_words[14] = s_words[15] = 0;
+}
+
+// Rank every exponent value by (count desc, value asc); write the plan of a
+// tensor of n elements; leave its histogram and ticket zeroed for reuse.
+template <int DT, int NT>
+__device__ void select_codebook(uint32_t *g_hist, uint32_t *g_ticket, uint64_t n, uint8_t *plan,
+                                uint32_t *ctl, uint32_t *s_cnt, uint8_t *s_cb, uint32_t *s_words) {
+    using C = PlanCfg<DT>;
+    const int tid = threadIdx.x;
+    for (int v = tid; v < C::kBins; v += NT) s_cnt[v] = __ldcg(g_hist + v);
+    __syncthreads();
+    for (int v = tid; v < C::kBins; v += NT) {
+        const uint32_t cv = s_cnt[v];
+        uint32_t rank = 0;
+#pragma unroll 8
+        for (int u = 0; u < C::kBins; ++u) {
+            const uint32_t cu = s_cnt[u];
+            rank += (cu > cv) | ((cu == cv) & (u < v));
+        }
+        if (rank < kCodes) s_cb[rank] = uint8_t(v);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint64_t sum = 0, covered = 0;
+        for (int v = 0; v < C::kBins; ++v) sum += s_cnt[v];
+        for (int c = 0; c < int(kCodes); ++c) covered += s_cnt[s_cb[c]];
+        if (sum != n) set_error(ctl, SZ_ERR_INTERNAL, 1);
+        make_plan_words(s_words, DT, n, n - covered, s_cb);
+    }
+    __syncthreads();
+    store_plan(plan, s_words);
+    for (int v = tid; v < C::kBins; v += NT) g_hist[v] = 0;
+    if (tid == 0) *g_ticket = 0;
+}
+
+template <int DT, int NT, int MAXB>
+__global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ PlanParams<MAXB> p) {
+    using C = PlanCfg<DT>;
+    extern __shared__ uint32_t s_cols[];  // C::kRows * NT packed counters
+    __shared__ uint32_t s_cnt[C::kBins];
+    __shared__ uint8_t s_cb[16];
+    __shared__ uint32_t s_words[16];
+    __shared__ uint32_t s_last;
+    const int tid = threadIdx.x;
+    uint32_t *col = s_cols + tid;
+
+    // Plans of empty tensors: codebook of the 15 smallest values, E = 0.
+    if (blockIdx.x == 0) {
+        for (int t = 0; t < p.T; ++t) {
+            if (p.n[t] != 0) continue;
+            if (tid == 0) {
+                uint8_t cb[kCodes];
+                for (int c = 0; c < int(kCodes); ++c) cb[c] = uint8_t(c);
+                make_plan_words(s_words, DT, 0, 0, cb);
+            }
+            __syncthreads();
+            store_plan(p.plans + 64 * size_t(t), s_words);
+            __syncthreads();
+        }
+    }
+
+    const uint64_t lo = p.total_items * blockIdx.x / gridDim.x;
+    const uint64_t hi = p.total_items * (blockIdx.x + 1) / gridDim.x;
+    if (lo >= hi) return;
+    for (int r = 0; r < C::kRows; ++r) s_cols[r * NT + tid] = 0;
+    __syncthreads();
+
+    int t = find_tensor<uint64_t, MAXB>(p.item_begin, p.T, lo);
+    uint64_t i = lo;
+    while (i < hi) {
+        while (p.item_begin[t + 1] <= i) ++t;  // skip tensors without items
+        const uint64_t i_end = min(hi, p.item_begin[t + 1]);
+        const uint64_t a = (i - p.item_begin[t]) * C::kItemElems;
+        const uint64_t b = min(p.n[t], (i_end - p.item_begin[t]) * C::kItemElems);
+        uint32_t *g_hist = p.hist + size_t(t) * 256;
+        // sub-ranges short enough that no 16-bit counter can overflow
+        constexpr uint64_t kSub = uint64_t(kMaxPerThread / C::kVecElems) * C::kVecElems * NT;
+        for (uint64_t s = a; s < b; s += kSub) {
+            count_range<DT, NT>(col, p.in[t], s, min(b, s + kSub));
+            flush_columns<DT, NT>(s_cols, g_hist);
+        }
+        // ticket: the CTA that completes the tensor's last item selects its codebook
+        if (tid == 0) {
+            const uint32_t items = uint32_t(i_end - i);
+            const uint32_t need = uint32_t(p.item_begin[t + 1] - p.item_begin[t]);
+            const uint32_t done = atomicAdd(p.ticket + t, items) + items;
+            s_last = (done == need);
+            __threadfence();
+        }
+        __syncthreads();
+        if (s_last) {
+            select_codebook<DT, NT>(g_hist, p.ticket + t, p.n[t], p.plans + 64 * size_t(t), p.ctl,
+                                    s_cnt, s_cb, s_words);
+            __syncthreads();
+        }
+        i = i_end;
+    }
+}
+
+template <int DT, int MAXB>
+sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
+    using C = PlanCfg<DT>;
+    constexpr int NT = kPlanThreads;
+    PlanParams<MAXB> p;
+    p.ctl = a.ctl;
+    p.hist = a.hist;
+    p.ticket = a.ticket;
+    p.plans = a.plans;
+    p.T = a.T;
+    p.item_begin[0] = 0;
+    for (int t = 0; t < a.T; ++t) {
+        p.in[t] = static_cast<const uint8_t *>(a.in[t]);
+        p.n[t] = a.n[t];
+        p.item_begin[t + 1] = p.item_begin[t] + cdiv(a.n[t], C::kItemElems);
+    }
+    p.total_items = p.item_begin[a.T];
+    const size_t smem = size_t(C::kRows) * NT * 4;
+    auto kern = plan_kernel<DT, NT, MAXB>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return SZ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess ||
+        per_sm < 1)
+        return SZ_ERR_CUDA;
+    uint64_t grid = uint64_t(a.num_sms) * per_sm;
+    if (p.total_items < grid) grid = p.total_items;
+    if (grid == 0) grid = 1;  // only empty tensors: block 0 writes their plans
+    kern<<<unsigned(grid), NT, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+}
+
+}  // namespace
+
+sz_status launch_plan(const PlanArgs &a, cudaStream_t stream) {
+    if (a.dtype == SZ_BF16)
+        return a.T <= kSmallBatch ? launch_plan_t<SZ_BF16, kSmallBatch>(a, stream)
+                                  : launch_plan_t<SZ_BF16, kLargeBatch>(a, stream);
+    return a.T <= kSmallBatch ? launch_plan_t<SZ_FP8_E5M2, kSmallBatch>(a, stream)
+                              : launch_plan_t<SZ_FP8_E5M2, kLargeBatch>(a, stream);
+}
+
+}  // namespace sz

@@ -1,0 +1,75 @@
+"""The C-ABI library loads and exports every function include/splitzip.h declares;
+host-only size functions agree with the oracle's closed form (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "splitzip.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sz_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_kv_cache_exp_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for must in ("sz_plan", "sz_encode", "sz_decode", "sz_compressed_size", "sz_plan_batched",
+                 "sz_encode_batched", "sz_decode_batched", "sz_last_device_status",
+                 "sz_workspace_bytes", "sz_max_compressed_size", "sz_status_string"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_names_match_header():
+    import fp8_kv_cache_exp_b200 as sz
+    for n in _declared():
+        assert hasattr(sz, n), n
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_host_sizes_match_oracle(lib, dtype):
+    lib.sz_stream_bytes.restype = ctypes.c_size_t
+    lib.sz_stream_bytes.argtypes = [ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64]
+    lib.sz_max_compressed_size.restype = ctypes.c_size_t
+    lib.sz_max_compressed_size.argtypes = [ctypes.c_int, ctypes.c_uint64]
+    rng = np.random.default_rng(0)
+    for n in [0, 1, 2, 4095, 4096, 4097, 8388608, (1 << 31), (1 << 32) - 1] + list(rng.integers(0, 1 << 30, 20)):
+        n = int(n)
+        for E in (0, n // 7, n):
+            assert lib.sz_stream_bytes(dtype, n, E) == oracle.compressed_size(dtype, n, E)
+        assert lib.sz_max_compressed_size(dtype, n) == oracle.compressed_size(dtype, n, n)
+    assert lib.sz_stream_bytes(9, 10, 0) == 0
+
+
+def test_workspace_sizes(lib):
+    import fp8_kv_cache_exp_b200 as sz
+    one = sz.sz_workspace_bytes(0, 8388608)
+    assert one == 256 + 1024 + 256 + 8 * 2048
+    assert sz.sz_workspace_bytes_batched(0, [8388608] * 64) == 256 + 64 * 1024 + 256 + 8 * 2048 * 64
+    assert sz.sz_workspace_bytes_batched(0, [1] * 257) == 0
+
+
+def test_status_strings():
+    import fp8_kv_cache_exp_b200 as sz
+    assert sz.sz_status_string(0) == "ok"
+    assert "corrupt" in sz.sz_status_string(4)
+    assert sz.sz_status_string(99) == "unknown status"

@@ -1,0 +1,137 @@
+"""Full-size GPU parity on the measured workloads, in the benchmark's launch configuration
+(one batched launch per kernel).  Every tensor up to 1 GB is compared with the CPU
+oracle byte for byte; the 4 GB stress tensor, too large for the oracle in test time,
+is checked by properties that hold at any size (bitwise round trip on the device,
+codebook and escape count against a torch bincount/sort, closed-form size).
+"""
+import numpy as np
+import pytest
+import torch
+
+import kvgen
+import oracle
+from gpu_helpers import raw_of, sz
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _run_batch(dtype, xs):
+    """Plan, encode and decode a batch in one launch each; returns streams and decodes."""
+    m = sz()
+    ns = [m.numel_of(x, dtype) for x in xs]
+    ws = m.new_workspace(dtype, ns)
+    plans = m.new_plans(len(xs))
+    m.sz_plan_batched(dtype, xs, ws, plans)
+    totals = m.sz_compressed_sizes(plans)
+    outs = [torch.full((t,), 0xA5, dtype=torch.uint8, device="cuda") for t in totals]
+    m.sz_encode_batched(dtype, plans, xs, outs, ws)
+    decs = [torch.full_like(x.view(torch.uint8), 0xA5).view(x.dtype) for x in xs]
+    m.sz_decode_batched(dtype, outs, decs, ws)
+    st = m.sz_last_device_status(ws)
+    assert st == 0, m.sz_status_string(st)
+    return plans, outs, decs
+
+
+def _check_against_oracle(dtype, xs, outs, decs, plans=None):
+    stats = []
+    for i, (x, out, dec) in enumerate(zip(xs, outs, decs)):
+        assert torch.equal(x.view(torch.uint8), dec.view(torch.uint8)), "round trip differs at %d" % i
+        raw = raw_of(x)
+        ref = oracle.encode(dtype, raw)
+        got = out.cpu().numpy()
+        assert got.size == ref.size, (i, got.size, ref.size)
+        d = np.nonzero(got != ref)[0]
+        assert d.size == 0, ("tensor", i, "first differing byte", int(d[0]))
+        if plans is not None:
+            assert np.array_equal(plans[i].cpu().numpy(), ref[:64])
+        stats.append(raw.size / ref.size)
+    return stats
+
+
+def test_llama3_8b_one_batch():
+    cfg = kvgen.CONFIGS["llama3-8b"]
+    xs = kvgen.kv_batch(cfg, device="cuda")
+    plans, outs, decs = _run_batch(0, xs)
+    ratios = _check_against_oracle(0, xs, outs, decs, plans)
+    assert min(ratios) > 1.25 and max(ratios) <= 4 / 3
+
+
+def test_llama3_8b_per_layer_equals_batch():
+    m = sz()
+    cfg = kvgen.CONFIGS["llama3-8b"]
+    xs = kvgen.kv_batch(cfg, device="cuda")
+    _, batch_outs, _ = _run_batch(0, xs)
+    for layer in range(cfg.layers):
+        pair = xs[2 * layer: 2 * layer + 2]
+        _, outs, decs = _run_batch(0, pair)
+        for j in range(2):
+            assert torch.equal(outs[j], batch_outs[2 * layer + j]), layer
+            assert torch.equal(decs[j].view(torch.uint8), pair[j].view(torch.uint8))
+
+
+@pytest.mark.parametrize("layer", [0, 31, 63])
+def test_qwen3_32b_layer(layer):
+    cfg = kvgen.CONFIGS["qwen3-32b"]
+    xs = [kvgen.kv_tensor(cfg, layer, kv, device="cuda") for kv in (0, 1)]
+    plans, outs, decs = _run_batch(0, xs)
+    _check_against_oracle(0, xs, outs, decs, plans)
+
+
+@pytest.mark.parametrize("size_index", [0, 1])
+@pytest.mark.parametrize("rare_index", range(len(kvgen.STRESS_RARE_PERCENT)))
+def test_stress_small(size_index, rare_index):
+    n = kvgen.STRESS_SIZES[size_index]
+    p = kvgen.STRESS_RARE_PERCENT[rare_index]
+    x = kvgen.stress_tensor(n, p, 4_000_000 + kvgen.stress_case(size_index, rare_index), device="cuda")
+    plans, outs, decs = _run_batch(0, [x])
+    _check_against_oracle(0, [x], outs, decs, plans)
+
+
+@pytest.mark.parametrize("rare_index", [2, 4])
+def test_stress_1gb(rare_index):
+    n = kvgen.STRESS_SIZES[2]
+    p = kvgen.STRESS_RARE_PERCENT[rare_index]
+    x = kvgen.stress_tensor(n, p, 4_000_000 + kvgen.stress_case(2, rare_index), device="cuda")
+    plans, outs, decs = _run_batch(0, [x])
+    _check_against_oracle(0, [x], outs, decs, plans)
+
+
+def _torch_codebook(x: torch.Tensor):
+    """(codebook, E) by torch.bincount + sort: (count desc, value asc)."""
+    w = x.view(torch.int16)
+    cnt = torch.zeros(256, dtype=torch.int64, device=x.device)
+    step = 1 << 28
+    for lo in range(0, w.numel(), step):
+        e = (w[lo: lo + step].to(torch.int32) >> 7) & 0xFF
+        cnt += torch.bincount(e, minlength=256)
+    key = cnt * 256 + (255 - torch.arange(256, device=x.device))
+    order = torch.argsort(key, descending=True)
+    cb = order[:15]
+    return cb.cpu().numpy().astype(np.uint8), int(x.numel() - cnt[cb].sum().item())
+
+
+def test_stress_4gb_properties():
+    m = sz()
+    n = kvgen.STRESS_SIZES[3]
+    x = kvgen.stress_tensor(n, 1, 4_000_000 + kvgen.stress_case(3, 1), device="cuda")
+    plans, outs, decs = _run_batch(0, [x])
+    assert torch.equal(decs[0].view(torch.uint8), x.view(torch.uint8))
+    hdr = plans[0].cpu().numpy()
+    cb, E = _torch_codebook(x)
+    assert np.array_equal(hdr[24:39], cb)
+    assert int(np.frombuffer(hdr[16:24].tobytes(), np.uint64)[0]) == E
+    assert outs[0].numel() == oracle.compressed_size(0, n, E)
+    # escapes: a sample of elements checked one by one against the codebook
+    s = outs[0]
+    nb = (n + 4095) // 4096
+    offs = s[64: 64 + 4 * (nb + 1)].view(torch.int32).to(torch.int64)
+    assert int(offs[0]) == 0 and int(offs[-1]) == E
+    assert bool((offs[1:] >= offs[:-1]).all())
+
+
+def test_qwen3_30b_a3b_e5m2_batch():
+    cfg = kvgen.CONFIGS["qwen3-30b-a3b-e5m2"]
+    xs = kvgen.kv_batch(cfg, device="cuda")
+    plans, outs, decs = _run_batch(1, xs)
+    ratios = _check_against_oracle(1, xs, outs, decs, plans)
+    assert max(ratios) <= 8 / 7 and min(ratios) > 1.10

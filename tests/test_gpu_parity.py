@@ -1,0 +1,122 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle, bit for bit.
+
+Small and ragged sizes span several 4096-element tiles and a partial last tile;
+the plan (= stream header), the whole compressed stream and the decoded tensor
+must equal the oracle's exactly (no tolerance: every step is integer work).
+"""
+import numpy as np
+import pytest
+import torch
+
+import kvgen
+import oracle
+import oracle_pins
+from gpu_helpers import check_parity, from_raw, gpu_decode, gpu_encode, raw_of, sz
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = (1, 2, 3, 7, 8, 9, 15, 16, 17, 255, 256, 257, 4095, 4096, 4097, 8191, 8193, 12289,
+          65536 + 5, (1 << 20) + 3)
+
+
+@pytest.mark.parametrize("kv", [0, 1], ids=["K", "V"])
+def test_phi2_layer(kv):
+    x = kvgen.kv_tensor(kvgen.CONFIGS["phi2"], 0, kv)
+    check_parity(0, raw_of(x))
+
+
+@pytest.mark.parametrize("dtype", [0, 1], ids=["bf16", "e5m2"])
+@pytest.mark.parametrize("n", RAGGED)
+def test_ragged_kvlike(dtype, n):
+    rng = np.random.default_rng(n)
+    check_parity(dtype, oracle_pins._kvlike(rng, n, dtype))
+
+
+@pytest.mark.parametrize("dtype", [0, 1], ids=["bf16", "e5m2"])
+@pytest.mark.parametrize("n", (1, 17, 4097, 50001))
+def test_ragged_uniform_bits(dtype, n):
+    rng = np.random.default_rng(100 + n)
+    check_parity(dtype, rng.integers(0, 256, n * (2 if dtype == 0 else 1)).astype(np.uint8))
+
+
+def test_exhaustive_bf16_patterns():
+    allp = np.arange(65536, dtype=np.uint32).astype("<u2")
+    rng = np.random.default_rng(0)
+    for x in (allp, allp[rng.permutation(allp.size)], np.repeat(allp, 3)):
+        check_parity(0, x.view(np.uint8))
+
+
+def test_exhaustive_e5m2_patterns():
+    allp = np.arange(256, dtype=np.uint32).astype(np.uint8)
+    rng = np.random.default_rng(0)
+    for x in (allp, allp[rng.permutation(allp.size)], np.repeat(allp, 17), np.tile(allp, 4099)):
+        check_parity(1, x)
+
+
+def test_special_cases():
+    check_parity(0, np.zeros(2 * 10000, np.uint8))                              # all +0.0
+    check_parity(0, np.full(9999, 0x8000, "<u2").view(np.uint8))                # all -0.0
+    check_parity(1, np.zeros(10001, np.uint8))
+    e = np.tile(np.arange(100, 116), 1024)                                      # 16 equal exponents
+    np.random.default_rng(1).shuffle(e)
+    check_parity(0, (e << 7).astype("<u2").view(np.uint8))
+    rng = np.random.default_rng(2)                                              # <= 15 distinct
+    vals = rng.choice(256, size=9, replace=False)
+    check_parity(0, ((rng.choice(vals, 20000) << 7) | rng.integers(0, 128, 20000)).astype("<u2").view(np.uint8))
+
+
+def test_golden_streams_on_gpu():
+    for path in oracle_pins.golden_files():
+        dtype, raw, expect = oracle_pins.load_golden(path)
+        plan, stream = gpu_encode(dtype, from_raw(raw, dtype))
+        assert np.array_equal(stream, expect), path
+        n = raw.size // (2 if dtype == 0 else 1)
+        assert np.array_equal(gpu_decode(dtype, expect, n), raw), path
+
+
+def test_empty_tensor():
+    m = sz()
+    for dtype in (0, 1):
+        ref = oracle.encode(dtype, np.zeros(0, np.uint8))
+        x = torch.empty(0, dtype=torch.bfloat16 if dtype == 0 else torch.float8_e5m2, device="cuda")
+        plan, stream = gpu_encode(dtype, x)
+        assert np.array_equal(stream, ref) and stream.size == 256
+
+
+def test_batched_matches_single():
+    """One launch per kernel over tensors of mixed sizes (empty ones included)."""
+    m = sz()
+    rng = np.random.default_rng(9)
+    for dtype in (0, 1):
+        sizes = [4096 * 3 + 17, 0, 1, 65536, 100003, 0, 4096, 777]
+        raws = [oracle_pins._kvlike(rng, n, dtype) for n in sizes]
+        xs = [from_raw(r, dtype) for r in raws]
+        ws = m.new_workspace(dtype, sizes)
+        plans = m.new_plans(len(xs))
+        m.sz_plan_batched(dtype, xs, ws, plans)
+        totals = m.sz_compressed_sizes(plans)
+        outs = [torch.full((m.sz_max_compressed_size(dtype, n),), 0xA5, dtype=torch.uint8, device="cuda")
+                for n in sizes]
+        m.sz_encode_batched(dtype, plans, xs, outs, ws)
+        decs = [torch.full_like(x.view(torch.uint8), 0xA5) for x in xs]
+        m.sz_decode_batched(dtype, [o[:t] for o, t in zip(outs, totals)],
+                            [d.view(x.dtype) for d, x in zip(decs, xs)], ws)
+        assert m.sz_last_device_status(ws) == 0
+        for raw, out, tot, dec in zip(raws, outs, totals, decs):
+            ref = oracle.encode(dtype, raw)
+            assert tot == ref.size
+            assert np.array_equal(out[:tot].cpu().numpy(), ref)
+            assert np.array_equal(dec.cpu().numpy(), raw)
+
+
+def test_workspace_reuse_is_deterministic():
+    m = sz()
+    x = kvgen.kv_tensor(kvgen.CONFIGS["phi2"], 0, 1).cuda()
+    ws = m.new_workspace(0, [x.numel()])
+    first = gpu_encode(0, x, ws)[1]
+    for _ in range(3):
+        assert np.array_equal(gpu_encode(0, x, ws)[1], first)
+    # a different batch through the same workspace, then the single tensor again
+    y = x.view(-1)[: 4096 * 5]
+    gpu_encode(0, y, ws)
+    assert np.array_equal(gpu_encode(0, x, ws)[1], first)
