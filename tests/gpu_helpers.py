@@ -24,8 +24,11 @@ def raw_of(x: torch.Tensor) -> np.ndarray:
 
 
 def from_raw(raw: np.ndarray, dtype: int, device="cuda") -> torch.Tensor:
+    tdt = torch.bfloat16 if dtype == 0 else torch.float8_e5m2
+    if raw.size == 0:
+        return torch.empty(0, dtype=tdt, device=device)
     t = torch.from_numpy(np.ascontiguousarray(raw).copy()).to(device)
-    return t.view(torch.bfloat16) if dtype == 0 else t.view(torch.float8_e5m2)
+    return t.view(tdt)
 
 
 POISON = 0xA5
