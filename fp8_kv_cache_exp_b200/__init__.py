@@ -5,7 +5,7 @@ Argument marshalling only: the functions below have the names of the C ABI in
 include/splitzip.h and pass torch tensors' device pointers and the current CUDA
 stream to it.  Every step of the codec runs in the library's CUDA kernels.
 Importing this package loads libsplitzip.so and raises ImportError if it has not
-been built (python -m fp8_kv_cache_exp_b200.build); there is no other path.
+been built (python fp8_kv_cache_exp_b200/build.py); there is no other path.
 """
 import ctypes
 import os
@@ -17,7 +17,7 @@ __all__ = [
     "sz_status_string", "sz_workspace_bytes", "sz_workspace_bytes_batched", "sz_stream_bytes",
     "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
     "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched", "sz_decode",
-    "sz_decode_batched", "sz_last_device_status", "dtype_of", "elem_bytes", "numel_of",
+    "sz_decode_batched", "sz_last_device_status", "sz_encode_noalloc", "dtype_of", "elem_bytes", "numel_of",
     "new_workspace", "new_plans",
 ]
 
@@ -37,13 +37,14 @@ SZ_ERR_INTERNAL = 8
 SZ_HEADER_BYTES = 64
 SZ_BLOCK_ELEMS = 4096
 SZ_MAX_BATCH = 256
+SZ_NOALLOC_MAX_ELEMS = 1 << 27
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitzip.so")
 
 
 def _load():
     if not os.path.exists(lib_path):
-        raise ImportError("libsplitzip.so is not built (%s); run: python -m fp8_kv_cache_exp_b200.build"
+        raise ImportError("libsplitzip.so is not built (%s); run: python fp8_kv_cache_exp_b200/build.py"
                           % lib_path)
     L = ctypes.CDLL(lib_path)
     vp, u64, sz, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_int
@@ -64,6 +65,7 @@ def _load():
         "sz_decode": (i32, [i32, vp, sz, vp, u64, vp, sz, vp]),
         "sz_decode_batched": (i32, [i32, i32, pvp, psz, pvp, pu64, vp, sz, vp]),
         "sz_last_device_status": (i32, [vp, vp]),
+        "sz_encode_noalloc": (i32, [i32, vp, vp, u64, vp, sz, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(L, name)
@@ -224,3 +226,12 @@ def sz_decode_batched(dtype: int, comps, outs, ws: torch.Tensor, comp_bytes=None
 def sz_last_device_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronise; return (and clear) the workspace's device error word."""
     return int(lib.sz_last_device_status(_p(ws), _stream(stream)))
+
+
+def sz_encode_noalloc(dtype: int, plan: torch.Tensor, x: torch.Tensor, out: torch.Tensor,
+                      status: torch.Tensor = None, stream=None):
+    """Encode with the library's own scratch (no workspace argument); `status`, if given,
+    is a device int32 tensor that receives the call's device error word."""
+    _check(lib.sz_encode_noalloc(dtype, _p(plan), _p(x), numel_of(x, dtype), _p(out), out.nbytes,
+                                 _p(status) if status is not None else None, _stream(stream)),
+           "sz_encode_noalloc")

@@ -1,6 +1,7 @@
 """Build libsplitzip.so (the CUDA library behind the C ABI) in-tree for sm_100a.
 
-Usage: python -m fp8_kv_cache_exp_b200.build [--force]
+Usage: python fp8_kv_cache_exp_b200/build.py [--force]
+(run it by path: importing the package itself loads the library it builds)
 """
 import glob
 import os

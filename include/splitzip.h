@@ -170,6 +170,36 @@ sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,
 /* Synchronise the stream, return the device error word of d_ws and clear it. */
 sz_status sz_last_device_status(void *d_ws, cudaStream_t stream);
 
+/* Largest n accepted by sz_encode_noalloc (2^27 elements: 32768 tiles). */
+#define SZ_NOALLOC_MAX_ELEMS (1ull << 27)
+
+/* Encode without a caller-provided workspace.  The paper has no counterpart:
+ * this is a convenience of this library.
+ *
+ * For callers that cannot allocate device memory where they encode -- for
+ * example an engine that reserves all of the GPU's memory for its KV pool at
+ * start-up and hands the codec only the tensor, the destination buffer and a
+ * stream.  The call runs the same kernel as sz_encode on a scratch area held
+ * by the library: a static device array of 262,400 bytes (enough for
+ * SZ_NOALLOC_MAX_ELEMS elements) that every GPU which loads the library keeps
+ * until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine; it enqueues a memset of the scratch it uses, the encode
+ * kernel and, if d_status is not NULL, a 4-byte device-to-device copy.
+ *
+ * Arguments are those of sz_encode; d_status (device, may be NULL) receives
+ * the call's device error word (SZ_OK or a device-found error) once the
+ * stream reaches it.  n > SZ_NOALLOC_MAX_ELEMS returns SZ_ERR_BUFFER_TOO_SMALL
+ * at once, with nothing enqueued.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call on a device shares the one scratch
+ * array, which keeps the previous call's contents (the call clears what must
+ * start at zero): calls whose work overlaps on the GPU -- on different
+ * streams, or from different threads -- race and must not be issued. */
+sz_status sz_encode_noalloc(sz_dtype dtype, const sz_plan_t *d_plan, const void *d_in, uint64_t n,
+                            void *d_out, size_t out_cap, uint32_t *d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,8 +21,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from fp8_kv_cache_exp_b200 import build
-    path = build.build()
+    import __graft_entry__
+    path = __graft_entry__._build_module().build()
     return ctypes.CDLL(path)
 
 
