@@ -120,34 +120,48 @@ struct PlanParams {
     uint64_t item_begin[MAXB + 1];  // prefix over tensors of ceil(n / item elements)
 };
 
+// Encode and decode work in chunks: up to kMaxChunkBlocks consecutive
+// 4096-element blocks of one tensor.  One look-back status word per chunk.
+constexpr int kMaxChunkLog2 = 4;
+constexpr int kMaxChunkBlocks = 1 << kMaxChunkLog2;
+
 template <int MAXB>
 struct EncodeParams {
     uint32_t *ctl;
-    unsigned long long *status;  // one look-back word per global tile
+    unsigned long long *status;  // one look-back word per global chunk
     const uint8_t *plans;
-    uint32_t total_tiles;
-    uint32_t total_jobs;         // tiles + empty tensors
+    uint32_t total_chunks;
+    uint32_t total_jobs;         // chunks + empty tensors
     int T;
     int n_empty;
+    int chunk_log2;              // blocks per chunk = 1 << chunk_log2
     const uint8_t *in[MAXB];
     uint8_t *out[MAXB];
     uint64_t n[MAXB];
     uint64_t cap[MAXB];
-    uint32_t tile_begin[MAXB + 1];
+    uint32_t chunk_begin[MAXB + 1];  // prefix over tensors of their chunk counts
     uint16_t empty[MAXB];
 };
 
 template <int MAXB>
 struct DecodeParams {
     uint32_t *ctl;
-    uint32_t total_tiles;
+    uint32_t total_blocks;
     int T;
     const uint8_t *comp[MAXB];
     uint64_t comp_bytes[MAXB];
     uint8_t *out[MAXB];
     uint64_t n[MAXB];
-    uint32_t tile_begin[MAXB + 1];
+    uint32_t block_begin[MAXB + 1];  // prefix over tensors of their 4096-element blocks
 };
+
+// Blocks per chunk for a launch: the largest power of two (<= kMaxChunkBlocks)
+// that still leaves at least two chunks per resident CTA.
+inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_ctas) {
+    int lg = kMaxChunkLog2;
+    while (lg > 0 && (total_blocks >> lg) < 2 * resident_ctas) --lg;
+    return lg;
+}
 
 // ---------------------------------------------------------- device helpers
 
@@ -178,6 +192,61 @@ __device__ inline uint32_t ld_relaxed_u32(const uint32_t *p) {
     return v;
 }
 
+// ------------------------------------------------ bulk copies and mbarriers
+// One-dimensional bulk copies global -> shared (the TMA engine, no tensor map),
+// completed on an mbarrier by transaction bytes.  Addresses and sizes must be
+// multiples of 16 bytes.  Every wait is bounded.
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the bulk-copy engine.
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's earlier shared-memory accesses before later bulk copies.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of the given parity to complete; false after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
 // Index t with begin[t] <= x < begin[t+1] (begin non-decreasing, begin[0] = 0).
 template <typename U, int MAXB>
 __device__ inline int find_tensor(const U (&begin)[MAXB + 1], int T, U x) {
@@ -187,6 +256,37 @@ __device__ inline int find_tensor(const U (&begin)[MAXB + 1], int T, U x) {
         if (begin[mid] <= x) lo = mid; else hi = mid;
     }
     return lo;
+}
+
+// Exclusive prefix of c over the lanes of a warp; *total receives the warp's
+// sum.  When no lane has c > 1 (escapes are rare) the prefix is a popcount of
+// the lanes below with c = 1; otherwise a shuffle scan.
+__device__ __forceinline__ uint32_t warp_exclusive_prefix(uint32_t c, uint32_t *total) {
+    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+    if (any == 0) {
+        *total = 0;
+        return 0;
+    }
+    const int lane = threadIdx.x & 31;
+    if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+        *total = __popc(any);
+        return __popc(any & ((1u << lane) - 1u));
+    }
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    *total = __shfl_sync(0xffffffffu, x, 31);
+    return x - c;
+}
+
+// Nibble flags of the escape code 15 among 8 packed 4-bit codes: bit 4j set
+// when code j is 15.
+__device__ __forceinline__ uint32_t escape_nibbles(uint32_t cw) {
+    const uint32_t t = cw & (cw >> 1);
+    return t & (t >> 2) & 0x11111111u;
 }
 
 // Exclusive prefix sum over the CTA (NT threads); *total receives the sum.

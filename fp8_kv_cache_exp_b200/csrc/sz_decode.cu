@@ -2,16 +2,23 @@
 //
 // SplitZip project page, FAQ "Is SplitZip lossy?": decoded tensors are
 // bitwise identical to the originals; FAQ "How can I reduce KV cache transfer
-// time ...": decompression runs on the decode GPU.  One CTA decodes one
-// 4096-element tile, independently of every other tile (the stored per-block
-// escape offsets make decode a pure gather):
-//   1. plane and code loads (issued before the header check: the host has
-//      already checked that the buffer holds the smallest stream for n);
-//   2. header and offsets checks -- a stream that fails one sets
-//      SZ_ERR_CORRUPT_STREAM and the tile writes nothing;
-//   3. escape ranks by a CTA prefix sum; the count must match the tile's
-//      offsets; the code -> exponent map is a 16-byte shared-memory table;
-//   4. elements reassembled with byte permutes and written with 16-byte stores.
+// time ...": decompression runs on the decode GPU.  The stored per-block
+// escape offsets make decode a pure gather with no dependency between blocks,
+// so one warp decodes one 4096-element block on its own, with no CTA barrier:
+//   - every warp owns a contiguous range of the launch's blocks, and checks a
+//     tensor's header (and builds its code-pair table) when it reaches it; a
+//     stream that fails a check sets SZ_ERR_CORRUPT_STREAM and is not written;
+//   - the block's code and plane bytes (6 KB BF16, 3.5 KB E5M2) arrive by bulk
+//     copy into one of the warp's two shared-memory stages while the warp
+//     decodes the previous block (waits are bounded); the next block's
+//     offsets-table entries and first 32 escape bytes are prefetched into
+//     registers the same way;
+//   - per 256-element (BF16) or 512-element (E5M2) step: each code byte (two
+//     4-bit codes) selects a pre-spread exponent pair from a 256-entry shared
+//     table; escape ranks come from a warp prefix of per-lane counts and the
+//     escape bytes from a shuffle; the elements are reassembled with byte
+//     permutes and integer multiply-adds and written with 16-byte stores
+//     (512 contiguous bytes per warp instruction).
 #include "sz_common.cuh"
 #include "sz_internal.h"
 
@@ -20,221 +27,465 @@ namespace sz {
 namespace {
 
 constexpr int NT = kTileThreads;
+constexpr int NW = NT / 32;
+constexpr uint32_t kStageBytes = 1536;                // a quarter block's codes and planes (BF16 size)
+constexpr int kStages = 4;                            // ring of quarter-block stages per warp
+constexpr uint64_t kWaitLimitNs = 1000000000ull;      // 1 s
 
-// Load `nbytes` (<= 8) bytes at p into (lo, hi), byte by byte.
-__device__ __forceinline__ void load_bytes(const uint8_t *p, int nbytes, uint32_t &lo, uint32_t &hi) {
-    lo = hi = 0;
+template <int DT>
+struct DGeo {
+    static constexpr int LE = (DT == SZ_BF16) ? 8 : 16;   // elements per lane per step
+    static constexpr int IT = int(kBlock) / (32 * LE);     // steps per block
+    static constexpr int QIT = IT / 4;                     // steps per quarter block
+    // quarter-block stage layout: codes, then plane a, then plane b
+    static constexpr uint32_t kCodeBytes = 512;
+    static constexpr uint32_t kABytes = (DT == SZ_BF16) ? 1024 : 128;
+    static constexpr uint32_t kBBytes = (DT == SZ_BF16) ? 0 : 256;
+    static constexpr uint32_t kA = kCodeBytes, kB = kCodeBytes + kABytes;
+    static constexpr uint32_t kBytes = kCodeBytes + kABytes + kBBytes;
+};
+
+struct alignas(128) WarpSmem {
+    uint8_t stage[kStages][kStageBytes];
+    uint32_t tab[256];       // code byte -> pre-spread exponent pair
+    uint64_t bar[kStages];   // one mbarrier per stage
+};
+
+// One lane's share of one step: codes and planes.
+struct DFrag {
+    uint32_t c0, c1;  // nibble codes (BF16: c0 only)
+    uint32_t a, b;    // BF16: sm bytes 0-3, 4-7 ; E5M2: 16 sign bits, 16 x 2 mantissa bits
+};
+
+// Per-warp decode state for the tensor it is working on.
+struct WarpStream {
+    int t;                        // tensor, -1 if none yet
+    bool ok;                      // header passed every check
+    uint32_t nb;                  // 4096-element blocks
+    uint64_t n, E;
+    uint64_t code, pa, pb, esc;   // section offsets in the stream
+};
+
+// Step `it` (within a quarter block) from a shared-memory stage.
+template <int DT>
+__device__ __forceinline__ DFrag read_stage(const uint8_t *st, int it) {
+    const int lane = threadIdx.x & 31;
+    DFrag f;
+    if constexpr (DT == SZ_BF16) {
+        f.c0 = *reinterpret_cast<const uint32_t *>(st + it * 128 + lane * 4);
+        f.c1 = 0;
+        const uint2 s = *reinterpret_cast<const uint2 *>(st + DGeo<DT>::kA + it * 256 + lane * 8);
+        f.a = s.x;
+        f.b = s.y;
+    } else {
+        const uint2 c = *reinterpret_cast<const uint2 *>(st + it * 256 + lane * 8);
+        f.c0 = c.x;
+        f.c1 = c.y;
+        f.a = *reinterpret_cast<const uint16_t *>(st + DGeo<DT>::kA + it * 64 + lane * 2);
+        f.b = *reinterpret_cast<const uint32_t *>(st + DGeo<DT>::kB + it * 128 + lane * 4);
+    }
+    return f;
+}
+
+__device__ __forceinline__ uint32_t load_le(const uint8_t *p, int nbytes) {
+    uint32_t v = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j < nbytes) {
-            const uint32_t b = p[j];
-            if (j < 4) lo |= b << (8 * j); else hi |= b << (8 * (j - 4));
+    for (int j = 0; j < 4; ++j)
+        if (j < nbytes) v |= uint32_t(p[j]) << (8 * j);
+    return v;
+}
+
+// Step `it` of a partial block straight from global memory: only `valid`
+// (< LE) elements of this lane exist.
+template <int DT>
+__device__ __forceinline__ DFrag read_partial(const uint8_t *comp, const WarpStream &ws, uint64_t blk,
+                                              int it, int valid) {
+    DFrag f = {0, 0, 0, 0};
+    if (valid <= 0) return f;
+    const int lane = threadIdx.x & 31;
+    const uint64_t e0 = blk * kBlock + uint64_t(it) * 32 * DGeo<DT>::LE + uint64_t(lane) * DGeo<DT>::LE;
+    const uint8_t *cd = comp + ws.code + e0 / 2;
+    const int cbytes = (valid + 1) / 2;
+    f.c0 = load_le(cd, cbytes < 4 ? cbytes : 4);
+    if (cbytes > 4) f.c1 = load_le(cd + 4, cbytes - 4);
+    if constexpr (DT == SZ_BF16) {
+        const uint8_t *sm = comp + ws.pa + e0;
+        f.a = load_le(sm, valid < 4 ? valid : 4);
+        if (valid > 4) f.b = load_le(sm + 4, valid - 4);
+    } else {
+        f.a = load_le(comp + ws.pa + e0 / 8, (valid + 7) / 8);
+        f.b = load_le(comp + ws.pb + e0 / 4, (valid + 3) / 4);
+    }
+    // codes of elements past n are ignored
+    if (valid < 8) {
+        f.c0 &= (1u << (4 * valid)) - 1u;
+        f.c1 = 0;
+    } else if (valid < 16) {
+        f.c1 &= (valid == 8) ? 0u : ((1u << (4 * (valid - 8))) - 1u);
+    }
+    return f;
+}
+
+// Check tensor t's header with the warp; on success fill the code-pair table:
+// tab[b] = exponents of the two codes in byte b, pre-spread for reassembly
+// (BF16: e_even | e_odd << 16; E5M2: e_even | e_odd << 8); code 15 gives 0.
+template <int DT, int MAXB>
+__device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, int t, uint32_t *tab, WarpStream &ws) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t *comp = p.comp[t];
+    const uint32_t hw = lane < 12 ? reinterpret_cast<const uint32_t *>(comp)[lane] : 0u;
+    uint32_t w[12];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) w[i] = __shfl_sync(0xffffffffu, hw, i);
+    const uint64_t n = p.n[t];
+    const uint64_t hn = uint64_t(w[2]) | (uint64_t(w[3]) << 32);
+    const uint64_t E = uint64_t(w[4]) | (uint64_t(w[5]) << 32);
+    const uint64_t total = uint64_t(w[10]) | (uint64_t(w[11]) << 32);
+    const uint32_t cbw[4] = {w[6], w[7], w[8], w[9]};
+    bool ok = w[0] == kMagic && (w[1] & 0xFF00FFFFu) == (header_vtag(DT) & 0xFF00FFFFu) &&
+              ((w[1] >> 16) & 0xFFu) == uint32_t(DT) && hn == n && E <= n && (w[9] >> 24) == 0 &&
+              total == stream_layout(DT, n, E).total && total <= p.comp_bytes[t];
+    // codebook: 15 distinct values inside the exponent range
+    bool cb_ok = true;
+    if (lane < int(kCodes)) {
+        const uint32_t c = cb_byte(cbw, lane);
+        cb_ok = c < uint32_t(Dt<DT>::kBins);
+        for (int d = 0; d < lane; ++d) cb_ok = cb_ok && cb_byte(cbw, d) != c;
+    }
+    ok = __all_sync(0xffffffffu, ok && cb_ok);
+    if (!ok && lane == 0) {
+        const bool dtype_mismatch = w[0] == kMagic && ((w[1] >> 16) & 0xFFu) != uint32_t(DT);
+        set_error(p.ctl, dtype_mismatch ? SZ_ERR_UNSUPPORTED_DTYPE : SZ_ERR_CORRUPT_STREAM, uint32_t(t));
+    }
+    if (ok) {
+        for (int b = lane; b < 256; b += 32) {
+            const uint32_t c0 = b & 15, c1 = b >> 4;
+            const uint32_t e0 = c0 < kCodes ? cb_byte(cbw, int(c0)) : 0u;
+            const uint32_t e1 = c1 < kCodes ? cb_byte(cbw, int(c1)) : 0u;
+            tab[b] = (DT == SZ_BF16) ? (e0 | (e1 << 16)) : (e0 | (e1 << 8));
         }
+    }
+    __syncwarp();
+    const Layout L = stream_layout(DT, n, ok ? E : 0);
+    ws.t = t;
+    ws.ok = ok;
+    ws.nb = uint32_t(L.nb);
+    ws.n = n;
+    ws.E = E;
+    ws.code = L.code;
+    ws.pa = L.plane[0];
+    ws.pb = L.plane[1];
+    ws.esc = L.esc;
+}
+
+// Section offsets of a tensor's stream; they depend on n only.
+struct StreamGeo {
+    const uint8_t *comp;
+    uint64_t code, pa, pb;
+};
+
+template <int DT, int MAXB>
+__device__ __forceinline__ StreamGeo stream_geo(const DecodeParams<MAXB> &p, int t) {
+    const Layout L = stream_layout(DT, p.n[t], 0);
+    StreamGeo g;
+    g.comp = p.comp[t];
+    g.code = L.code;
+    g.pa = L.plane[0];
+    g.pb = L.plane[1];
+    return g;
+}
+
+// Lane 0 starts the bulk copies of quarter q of block blk into a stage.
+template <int DT>
+__device__ __forceinline__ void issue_quarter(uint8_t *st, uint64_t *bar, const StreamGeo &sg,
+                                              uint64_t blk, int q) {
+    using G = DGeo<DT>;
+    const uint64_t u = blk * 4 + q;  // quarter index within the tensor
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, G::kBytes);
+    bulk_g2s(st, sg.comp + sg.code + u * G::kCodeBytes, G::kCodeBytes, bar);
+    bulk_g2s(st + G::kA, sg.comp + sg.pa + u * G::kABytes, G::kABytes, bar);
+    if (G::kBBytes) bulk_g2s(st + G::kB, sg.comp + sg.pb + u * G::kBBytes, G::kBBytes, bar);
+}
+
+// Add escape exponent e of element j (of this lane's LE elements) into o.
+template <int DT>
+__device__ __forceinline__ void patch(uint32_t (&o)[4], uint32_t j, uint32_t e) {
+    uint32_t k, add;
+    if constexpr (DT == SZ_BF16) {
+        k = j >> 1;
+        add = e << (7 + 16 * (j & 1));
+    } else {
+        k = j >> 2;
+        add = e << (2 + 8 * (j & 3));
+    }
+    o[0] += (k == 0) ? add : 0u;
+    o[1] += (k == 1) ? add : 0u;
+    o[2] += (k == 2) ? add : 0u;
+    o[3] += (k == 3) ? add : 0u;
+}
+
+// Decode one step.  running: escapes of the block before this step (updated);
+// esc_reg: lane i holds the block's escape i (i < 32); esc_g: the block's
+// escapes in global memory; cnt: escapes the offsets table gives the block.
+template <int DT, bool PARTIAL>
+__device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab, uint8_t *dst,
+                                            int valid, uint32_t &running, uint32_t esc_reg,
+                                            const uint8_t *esc_g, uint32_t cnt, bool &bad) {
+    uint32_t o[4];
+    uint64_t m;  // escape flags of this lane's elements: bit 4j for element j
+    if constexpr (DT == SZ_BF16) {
+        const uint32_t cw = f.c0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t e2 = tab[(cw >> (8 * k)) & 0xFFu];
+            const uint32_t x = __byte_perm((k < 2) ? f.a : f.b, 0, (k & 1) ? 0x4342 : 0x4140);
+            o[k] = x + (x & 0x00800080u) * 0xFFu + (e2 << 7);
+        }
+        m = escape_nibbles(cw);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t cw = (k < 2) ? f.c0 : f.c1;
+            const uint32_t lo = tab[(cw >> (16 * (k & 1))) & 0xFFu];
+            const uint32_t hi = tab[(cw >> (16 * (k & 1) + 8)) & 0xFFu];
+            const uint32_t e4 = lo | (hi << 16);
+            const uint32_t s4 = (f.a >> (4 * k)) & 0xFu;
+            const uint32_t sgn = (s4 * 0x10204080u) & 0x80808080u;
+            const uint32_t m8 = (f.b >> (8 * k)) & 0xFFu;
+            const uint32_t mnt = (m8 | (m8 << 6) | (m8 << 12) | (m8 << 18)) & 0x03030303u;
+            o[k] = (sgn | mnt) + (e4 << 2);
+        }
+        m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
+    }
+    const uint32_t c = __popcll(m);
+    uint32_t tot;
+    const uint32_t prefix = warp_exclusive_prefix(c, &tot);
+    if (tot) {
+        const uint32_t maxc = __reduce_max_sync(0xffffffffu, c);
+        uint64_t mm = m;
+        for (uint32_t i = 0; i < maxc; ++i) {
+            const uint32_t r = running + prefix + i;
+            const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
+            if (i < c) {
+                const uint32_t j = uint32_t(__ffsll(mm) - 1) >> 2;  // element, in element order
+                mm &= mm - 1;
+                uint32_t e = 0;
+                if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
+                else bad = true;
+                if (DT == SZ_FP8_E5M2 && e >= 32u) bad = true;
+                patch<DT>(o, j, e & (Dt<DT>::kBins - 1));
+            }
+        }
+        running += tot;
+    }
+    if (!PARTIAL) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else if constexpr (DT == SZ_BF16) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < valid) reinterpret_cast<uint16_t *>(dst)[j] = uint16_t(o[j >> 1] >> (16 * (j & 1)));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < valid) dst[j] = uint8_t(o[j >> 2] >> (8 * (j & 3)));
     }
 }
 
+// Offsets-table entries of a block and their checks.
+struct BlockEsc {
+    uint32_t lo, hi;
+};
+
+__device__ __forceinline__ BlockEsc load_offsets(const uint8_t *comp, uint64_t blk) {
+    const uint32_t *tabw = reinterpret_cast<const uint32_t *>(comp + 64);
+    BlockEsc b;
+    b.lo = tabw[blk];
+    b.hi = tabw[blk + 1];
+    return b;
+}
+
+__device__ __forceinline__ bool offsets_ok(const BlockEsc &b, const WarpStream &ws, uint64_t blk) {
+    return b.lo <= b.hi && b.hi <= ws.E && b.hi - b.lo <= kBlock && (blk != 0 || b.lo == 0) &&
+           (blk + 1 != ws.nb || b.hi == ws.E);
+}
+
+__device__ __forceinline__ uint32_t load_escape_reg(const uint8_t *comp, const WarpStream &ws,
+                                                    const BlockEsc &b) {
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t cnt = b.hi >= b.lo ? b.hi - b.lo : 0u;
+    return (lane < cnt && b.hi <= ws.E) ? uint32_t(comp[ws.esc + b.lo + lane]) : 0u;
+}
+
+// The warp's quarter-block units in order; the producer side of its ring.
+template <int DT, int MAXB>
+struct QuarterFeed {
+    uint32_t g, g_end;  // block (launch-global) of the next unit to issue, end of range
+    int q, t;           // its quarter and tensor
+    StreamGeo sg;
+    uint32_t v;         // units issued so far
+
+    __device__ __forceinline__ void start(const DecodeParams<MAXB> &p, uint32_t b_lo, uint32_t b_hi, int t0) {
+        g = b_lo;
+        g_end = b_hi;
+        q = 0;
+        t = t0;
+        sg = stream_geo<DT, MAXB>(p, t);
+        v = 0;
+    }
+    // Issue the next unit into stage v % kStages (if it is part of a full
+    // block); returns the bit to set in the issued mask.
+    __device__ __forceinline__ uint32_t issue_next(const DecodeParams<MAXB> &p, WarpSmem &W) {
+        if (g >= g_end) return 0;
+        if (p.block_begin[t + 1] <= g) {
+            while (p.block_begin[t + 1] <= g) ++t;
+            sg = stream_geo<DT, MAXB>(p, t);
+        }
+        const uint64_t blk = g - p.block_begin[t];
+        const int st = int(v % kStages);
+        uint32_t bit = 0;
+        if ((blk + 1) * kBlock <= p.n[t]) {
+            if ((threadIdx.x & 31) == 0) issue_quarter<DT>(W.stage[st], &W.bar[st], sg, blk, q);
+            bit = 1u << st;
+        }
+        ++v;
+        if (++q == 4) {
+            q = 0;
+            ++g;
+        }
+        return bit;
+    }
+};
+
 template <int DT, int MAXB>
 __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
-    __shared__ uint32_t s_hdr[12];
-    __shared__ uint32_t s_off[2];
-    __shared__ uint32_t s_warp[NT / 32];
-    __shared__ uint32_t s_bad;
-    __shared__ uint8_t s_cb[16];
-    const int tid = threadIdx.x;
-    const uint32_t job = blockIdx.x;
-    const int t = find_tensor<uint32_t, MAXB>(p.tile_begin, p.T, job);
-    const uint32_t tile = job - p.tile_begin[t];
-    const uint64_t n = p.n[t];
-    const uint8_t *comp = p.comp[t];
-    uint8_t *out = p.out[t];
-    // the plane and code positions depend on n only (not on E)
-    const Layout L0 = stream_layout(DT, n, 0);
-    if (tid < 12) s_hdr[tid] = reinterpret_cast<const uint32_t *>(comp)[tid];
-    if (tid < 2) s_off[tid] = reinterpret_cast<const uint32_t *>(comp + 64)[tile + tid];
-    if (tid == 0) s_bad = 0;
+    using G = DGeo<DT>;
+    extern __shared__ __align__(128) uint8_t s_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WarpSmem &W = reinterpret_cast<WarpSmem *>(s_raw)[warp];
+    if (lane == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&W.bar[i], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
 
-    // ---- 1. loads
-    constexpr int G = (DT == SZ_BF16) ? 2 : 1;
-    constexpr int kGE = (DT == SZ_BF16) ? 8 : 16;
-    const uint64_t e_tile = uint64_t(tile) * kBlock;
-    uint64_t e0[G];
-    int valid[G];
-    uint32_t cw[G][2], pa[G], pb[G];  // codes; BF16: sm lo/hi ; E5M2: sign, mantissa
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        e0[g] = e_tile + uint64_t(g) * (kBlock / 2) + uint64_t(tid) * kGE;
-        valid[g] = n > e0[g] ? int(min(uint64_t(kGE), n - e0[g])) : 0;
-        cw[g][0] = cw[g][1] = pa[g] = pb[g] = 0;
-        if constexpr (DT == SZ_BF16) {
-            const uint8_t *cd = comp + L0.code + e0[g] / 2;
-            const uint8_t *sm = comp + L0.plane[0] + e0[g];
-            if (valid[g] == 8) {
-                cw[g][0] = __ldcs(reinterpret_cast<const unsigned int *>(cd));
-                const uint2 s = __ldcs(reinterpret_cast<const uint2 *>(sm));
-                pa[g] = s.x;
-                pb[g] = s.y;
-            } else if (valid[g] > 0) {
-                uint32_t unused;
-                load_bytes(cd, (valid[g] + 1) / 2, cw[g][0], unused);
-                load_bytes(sm, valid[g], pa[g], pb[g]);
+    // every warp owns a contiguous range of the launch's blocks
+    const uint64_t nwarps = uint64_t(gridDim.x) * NW;
+    const uint64_t gw = uint64_t(blockIdx.x) * NW + warp;
+    const uint32_t b_lo = uint32_t(uint64_t(p.total_blocks) * gw / nwarps);
+    const uint32_t b_hi = uint32_t(uint64_t(p.total_blocks) * (gw + 1) / nwarps);
+    if (b_lo >= b_hi) return;
+
+    int t = find_tensor<uint32_t, MAXB>(p.block_begin, p.T, b_lo);
+    QuarterFeed<DT, MAXB> feed;
+    feed.start(p, b_lo, b_hi, t);
+    uint32_t issued = 0;  // bit s: stage s holds an issued unit not yet waited for
+    uint32_t parity = 0;  // bit s: parity of stage s's next completion
+    for (int k = 0; k < kStages - 1; ++k) issued |= feed.issue_next(p, W);
+
+    WarpStream ws;
+    warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
+    uint64_t blk = b_lo - p.block_begin[t];
+    BlockEsc be = load_offsets(p.comp[t], blk);
+    uint32_t esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
+    uint32_t v = 0;  // units consumed
+
+    for (uint32_t g = b_lo; g < b_hi; ++g) {
+        const uint8_t *comp = p.comp[t];
+        const bool next_same = g + 1 < b_hi && g + 1 < p.block_begin[t + 1];
+        BlockEsc be_n = {0, 0};
+        if (next_same && ws.ok) be_n = load_offsets(comp, blk + 1);
+        uint32_t esc_n = 0;
+
+        const bool ok = ws.ok && offsets_ok(be, ws, blk);
+        const uint32_t cnt = ok ? be.hi - be.lo : 0u;
+        const uint8_t *esc_g = comp + ws.esc + be.lo;
+        uint8_t *out = p.out[t] + (blk * kBlock + uint64_t(lane) * G::LE) * Dt<DT>::kElemBytes;
+        const bool full = (blk + 1) * kBlock <= ws.n;
+        uint32_t running = 0;
+        bool bad = false, timed_out = false;
+        for (int q = 0; q < 4; ++q, ++v) {
+            issued |= feed.issue_next(p, W);
+            const int st = int(v % kStages);
+            if (issued & (1u << st)) {
+                timed_out = timed_out || !mbar_wait(&W.bar[st], (parity >> st) & 1u, kWaitLimitNs);
+                parity ^= 1u << st;
+                issued &= ~(1u << st);
             }
+            if (q == 1 && next_same && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
+            if (ok && !timed_out) {
+                if (full) {
+#pragma unroll
+                    for (int it = 0; it < G::QIT; ++it) {
+                        const DFrag f = read_stage<DT>(W.stage[st], it);
+                        decode_step<DT, false>(f, W.tab, out + (q * G::QIT + it) * 512, G::LE, running,
+                                               esc_reg, esc_g, cnt, bad);
+                    }
+                } else {
+                    for (int it = q * G::QIT; it < (q + 1) * G::QIT; ++it) {
+                        const int64_t e = int64_t(blk * kBlock) + int64_t(it) * 32 * G::LE + int64_t(lane) * G::LE;
+                        const int64_t left = int64_t(ws.n) - e;
+                        const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+                        const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
+                        decode_step<DT, true>(f, W.tab, out + it * 512, valid, running, esc_reg, esc_g, cnt, bad);
+                    }
+                }
+            }
+            __syncwarp();  // the stage just read may be refilled from here on
+        }
+        if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
+        if (lane == 0) {
+            if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, g);
+            else if (ws.ok && (!ok || bad)) set_error(p.ctl, SZ_ERR_CORRUPT_STREAM, g);
+        }
+        if (timed_out) return;  // a copy that never lands: stop this warp
+
+        // ---- advance
+        if (g + 1 >= b_hi) break;
+        if (next_same) {
+            ++blk;
+            be = be_n;
+            esc_reg = esc_n;
         } else {
-            const uint8_t *sg = comp + L0.plane[0] + e0[g] / 8;
-            const uint8_t *mt = comp + L0.plane[1] + e0[g] / 4;
-            const uint8_t *cd = comp + L0.code + e0[g] / 2;
-            if (valid[g] == 16) {
-                pa[g] = __ldcs(reinterpret_cast<const unsigned short *>(sg));
-                pb[g] = __ldcs(reinterpret_cast<const unsigned int *>(mt));
-                const uint2 c = __ldcs(reinterpret_cast<const uint2 *>(cd));
-                cw[g][0] = c.x;
-                cw[g][1] = c.y;
-            } else if (valid[g] > 0) {
-                uint32_t unused;
-                load_bytes(sg, (valid[g] + 7) / 8, pa[g], unused);
-                load_bytes(mt, (valid[g] + 3) / 4, pb[g], unused);
-                load_bytes(cd, (valid[g] + 1) / 2, cw[g][0], cw[g][1]);
-            }
-        }
-        // codes of elements past n are ignored
-        if (valid[g] < kGE) {
-            if (valid[g] <= 8) {
-                cw[g][0] &= (valid[g] == 8) ? 0xffffffffu : ((1u << (4 * valid[g])) - 1u);
-                cw[g][1] = 0;
-            } else {
-                cw[g][1] &= (1u << (4 * (valid[g] - 8))) - 1u;
-            }
+            while (p.block_begin[t + 1] <= g + 1) ++t;
+            warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
+            blk = 0;
+            be = load_offsets(p.comp[t], blk);
+            esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
         }
     }
-    __syncthreads();
-
-    // ---- 2. header and offsets checks
-    const Header H = load_header(reinterpret_cast<const uint8_t *>(s_hdr));
-    const uint64_t lo = s_off[0], hi = s_off[1];
-    bool ok = H.magic == kMagic && (H.vtag & 0xFF00FFFFu) == (header_vtag(DT) & 0xFF00FFFFu) &&
-              H.n == n && H.E <= n && (H.cbw[3] >> 24) == 0;
-    const bool dtype_ok = ((H.vtag >> 16) & 0xFFu) == uint32_t(DT);
-    ok = ok && dtype_ok;
-    const Layout L = stream_layout(DT, n, ok ? H.E : 0);
-    ok = ok && H.total == L.total && H.total <= p.comp_bytes[t];
-    ok = ok && lo <= hi && hi <= H.E && hi - lo <= kBlock;
-    ok = ok && (tile != 0 || lo == 0) && (uint64_t(tile) + 1 != L.nb || hi == H.E);
-    if (tid < int(kCodes)) {
-        const uint32_t c = cb_byte(H.cbw, tid);
-        bool cb_ok = c < uint32_t(Dt<DT>::kBins);
-        for (int d = 0; d < tid; ++d) cb_ok = cb_ok && cb_byte(H.cbw, d) != c;
-        s_cb[tid] = uint8_t(c);
-        if (!cb_ok) s_bad = 1;
-    }
-    if (tid == 15) s_cb[15] = 0;
-    __syncthreads();
-    if (!ok || s_bad) {
-        if (tid == 0) set_error(p.ctl, dtype_ok || H.magic != kMagic ? SZ_ERR_CORRUPT_STREAM
-                                                                     : SZ_ERR_UNSUPPORTED_DTYPE, job);
-        return;
-    }
-
-    // ---- 3. escape ranks
-    uint32_t emask[G];
-    uint32_t packed = 0;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        uint32_t bits = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t c = cw[g][h];
-            const uint32_t m = c & (c >> 1) & (c >> 2) & (c >> 3) & 0x11111111u;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bits |= ((m >> (4 * j)) & 1u) << (8 * h + j);
-        }
-        emask[g] = bits;
-        packed |= uint32_t(__popc(bits)) << (16 * g);
-    }
-    uint32_t total_packed;
-    const uint32_t before = block_exclusive_scan<NT>(packed, s_warp, &total_packed);
-    const uint32_t tile_escapes = (total_packed & 0xFFFFu) + (total_packed >> 16);
-    if (tile_escapes != hi - lo) {  // uniform across the CTA
-        if (tid == 0) set_error(p.ctl, SZ_ERR_CORRUPT_STREAM, job);
-        return;
-    }
-    const uint8_t *esc = comp + L.esc + lo;
-
-    // ---- 4. reassemble and store
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        if (valid[g] <= 0) continue;
-        uint32_t r = (g == 0) ? (before & 0xFFFFu) : (total_packed & 0xFFFFu) + (before >> 16);
-        uint32_t ex[kGE];
-#pragma unroll
-        for (int j = 0; j < kGE; ++j) ex[j] = s_cb[(cw[g][j >> 3] >> (4 * (j & 7))) & 0xFu];
-        uint32_t m = emask[g];
-        bool bad_esc = false;
-        while (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1;
-            const uint32_t e = esc[r++];
-            if (DT == SZ_FP8_E5M2 && e >= 32u) bad_esc = true;
-#pragma unroll
-            for (int q = 0; q < kGE; ++q)
-                if (q == j) ex[q] = e & (Dt<DT>::kBins - 1);
-        }
-        if (bad_esc) set_error(p.ctl, SZ_ERR_CORRUPT_STREAM, job);
-        uint32_t o[4];
-        if constexpr (DT == SZ_BF16) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t src = (k < 2) ? pa[g] : pb[g];
-                const uint32_t x = __byte_perm(src, 0, (k & 1) ? 0x4342 : 0x4140);
-                const uint32_t e2 = ex[2 * k] | (ex[2 * k + 1] << 16);
-                o[k] = (x & 0x007F007Fu) | ((x & 0x00800080u) << 8) | (e2 << 7);
-            }
-            uint8_t *dst = out + 2 * e0[g];
-            if (valid[g] == 8) {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (j < valid[g])
-                        reinterpret_cast<uint16_t *>(dst)[j] = uint16_t(o[j >> 1] >> (16 * (j & 1)));
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t s4 = (pa[g] >> (4 * k)) & 0xFu;
-                const uint32_t sgn = ((s4 * 0x00204081u) & 0x01010101u) << 7;
-                const uint32_t m8 = (pb[g] >> (8 * k)) & 0xFFu;
-                const uint32_t mnt = (m8 | (m8 << 6) | (m8 << 12) | (m8 << 18)) & 0x03030303u;
-                const uint32_t e4 = ex[4 * k] | (ex[4 * k + 1] << 8) | (ex[4 * k + 2] << 16) |
-                                    (ex[4 * k + 3] << 24);
-                o[k] = sgn | (e4 << 2) | mnt;
-            }
-            uint8_t *dst = out + e0[g];
-            if (valid[g] == 16) {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (j < valid[g]) dst[j] = uint8_t(o[j >> 2] >> (8 * (j & 3)));
-            }
-        }
-    }
+    // wait for copies still in flight before the warp's shared memory goes away
+    for (int st = 0; st < kStages; ++st)
+        if (issued & (1u << st)) mbar_wait(&W.bar[st], (parity >> st) & 1u, kWaitLimitNs);
 }
 
 template <int DT, int MAXB>
 sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
+    auto kern = decode_kernel<DT, MAXB>;
+    const size_t smem = sizeof(WarpSmem) * NW;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return SZ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess || per_sm < 1)
+        return SZ_ERR_CUDA;
     DecodeParams<MAXB> p;
     p.ctl = a.ctl;
     p.T = a.T;
-    p.tile_begin[0] = 0;
+    p.block_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
         p.comp[t] = static_cast<const uint8_t *>(a.comp[t]);
         p.comp_bytes[t] = a.comp_bytes[t];
         p.out[t] = static_cast<uint8_t *>(a.out[t]);
         p.n[t] = a.n[t];
-        p.tile_begin[t + 1] = p.tile_begin[t] + uint32_t(cdiv(a.n[t], kBlock));
+        p.block_begin[t + 1] = p.block_begin[t] + uint32_t(cdiv(a.n[t], kBlock));
     }
-    p.total_tiles = p.tile_begin[a.T];
-    if (p.total_tiles == 0) return SZ_OK;
-    decode_kernel<DT, MAXB><<<p.total_tiles, NT, 0, stream>>>(p);
+    p.total_blocks = p.block_begin[a.T];
+    if (p.total_blocks == 0) return SZ_OK;
+    // enough CTAs to fill the GPU, but no more warps than blocks
+    const uint64_t resident = uint64_t(a.num_sms) * per_sm;
+    const uint64_t need = cdiv(p.total_blocks, NW);
+    const uint64_t grid = need < resident ? need : resident;
+    kern<<<unsigned(grid), NT, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
 

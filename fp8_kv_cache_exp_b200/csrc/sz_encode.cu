@@ -2,20 +2,22 @@
 //
 // SplitZip project page, Abstract: sign and mantissa bits are kept exactly,
 // frequent exponents get fixed 4-bit codes, rare exponents go to a sparse
-// escape stream.  One CTA encodes one 4096-element tile:
-//   1. 16-byte loads of the tile, exponent -> code through a 256-entry
-//      shared-memory table built from the plan's codebook;
-//   2. sign|mantissa bytes (BF16) or sign bits + 2-bit mantissas (E5M2) and
-//      the 4-bit codes stored with 4-16 byte coalesced stores;
-//   3. escapes counted per thread, ranked by a CTA prefix sum, and staged in
-//      shared memory in element order;
-//   4. the tile's escape offset found by a single-pass decoupled look-back
-//      over the tiles of its tensor (tile ids taken from an atomic counter in
-//      launch order, so every predecessor is already running; every wait is
-//      bounded and reports SZ_ERR_TIMEOUT instead of hanging);
-//   5. staged escapes written contiguously at that offset; the tile's entry
-//      of the offsets table written; the tensor's last tile also writes the
-//      header, offsets[nb] and the zero padding between sections.
+// escape stream.  Persistent CTAs take chunks (up to 16 consecutive
+// 4096-element blocks of one tensor) in launch order from an atomic counter:
+//   1. each block: 16-byte loads (the next block prefetched), exponent -> code
+//      through a 256-entry shared table built from the plan's codebook,
+//      sign|mantissa bytes (BF16) or sign bits + 2-bit mantissas (E5M2) and
+//      4-bit codes written with coalesced 2-8 byte stores;
+//   2. escapes of each block ranked by a CTA prefix sum and staged in shared
+//      memory in element order, with the block's offset within the chunk;
+//   3. the chunk's escape offset found by a single-pass decoupled look-back
+//      over the chunks of its tensor: every chunk with a lower id is already
+//      claimed by a running CTA, a 128-chunk window is read per step, and the
+//      wait is bounded (SZ_ERR_TIMEOUT instead of a hang);
+//   4. the chunk's entries of the offsets table and its staged escapes written
+//      contiguously (a chunk whose escapes overflow the stage re-reads its
+//      input and writes them directly); the tensor's last chunk also writes
+//      the header, offsets[nb] and the zero padding between sections.
 #include "sz_common.cuh"
 #include "sz_internal.h"
 
@@ -24,56 +26,86 @@ namespace sz {
 namespace {
 
 constexpr int NT = kTileThreads;
+constexpr int NW = NT / 32;
+constexpr int kChunkBlocks = NW;                      // a chunk is one block per warp
+constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per block
+constexpr int kLookbackPerLane = 4;                   // status words per lane per step
 constexpr uint64_t kLookbackLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
-constexpr unsigned long long kFlagAgg = 1ull << 32;    // tile aggregate published
-constexpr unsigned long long kFlagInc = 2ull << 32;    // inclusive prefix published
+constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate published
+constexpr unsigned long long kFlagInc = 2ull << 32;   // inclusive prefix published
 
-struct TileShared {
+struct EncShared {
     uint32_t hdr[16];
-    uint32_t warp[NT / 32];
-    uint32_t excl;
-    uint8_t lut[256];
-    alignas(16) uint8_t esc[kBlock];
+    uint32_t cnt[kChunkBlocks];      // escapes of each block of the chunk
+    uint32_t blk_off[kChunkBlocks];  // escapes before each block, within the chunk
+    uint32_t job, excl;
+    uint8_t lut[256];                // exponent -> code
+    alignas(16) uint8_t esc[kChunkBlocks][kWarpStage];
 };
 
-// Decoupled look-back, run by warp 0.  Returns the number of escapes in the
-// tensor's tiles before `tile`; publishes this tile's aggregate at once and
-// its inclusive prefix when known.  Status word: epoch (30 bits) << 34 |
-// flag << 32 | value; words from earlier launches carry an older epoch and
-// read as "not published".
-__device__ uint32_t lookback(unsigned long long *st, uint32_t tile, uint32_t agg, uint32_t epoch,
+template <int DT>
+struct Geo {
+    static constexpr int LE = (DT == SZ_BF16) ? 8 : 16;    // elements per lane per step
+    static constexpr int IT = int(kBlock) / (32 * LE);      // steps per block
+    static constexpr int kAhead = 3;                        // steps of loads in flight
+};
+
+// Decoupled look-back, run by warp 0.  Returns the escapes in the tensor's
+// chunks before `chunk`; publishes this chunk's aggregate at once and its
+// inclusive prefix when known.  Status word: epoch (30 bits) << 34 |
+// flag << 32 | value; words of earlier launches carry an older epoch and read
+// as "not published".  Lane l reads positions 4l..4l+3 behind the cursor
+// (position 0 = nearest predecessor).
+__device__ uint32_t lookback(unsigned long long *st, uint32_t chunk, uint32_t agg, uint32_t epoch,
                              bool *timed_out) {
     const int lane = threadIdx.x & 31;
     const unsigned long long tag = (unsigned long long)(epoch & 0x3FFFFFFFu) << 34;
     *timed_out = false;
-    if (tile == 0) {
+    if (chunk == 0) {
         if (lane == 0) st_relaxed_u64(st, tag | kFlagInc | agg);
         return 0;
     }
-    if (lane == 0) st_relaxed_u64(st + tile, tag | kFlagAgg | agg);
+    if (lane == 0) st_relaxed_u64(st + chunk, tag | kFlagAgg | agg);
     uint32_t excl = 0;
-    int64_t j = int64_t(tile) - 1;  // nearest predecessor, read by lane 0
+    int64_t j = int64_t(chunk) - 1;
     uint64_t t0 = 0;
     uint32_t backoff = 32;
     while (true) {
-        const int64_t idx = j - lane;
-        uint32_t flag = 2, val = 0;  // before tile 0: a virtual inclusive 0
-        if (idx >= 0) {
-            const unsigned long long w = ld_relaxed_u64(st + idx);
-            flag = ((w >> 34) == (tag >> 34)) ? uint32_t(w >> 32) & 3u : 0u;
-            val = uint32_t(w);
+        uint32_t f[kLookbackPerLane], v[kLookbackPerLane];
+#pragma unroll
+        for (int q = 0; q < kLookbackPerLane; ++q) {
+            const int64_t idx = j - kLookbackPerLane * lane - q;
+            f[q] = 2;  // before chunk 0: a virtual inclusive prefix of 0
+            v[q] = 0;
+            if (idx >= 0) {
+                const unsigned long long w = ld_relaxed_u64(st + idx);
+                f[q] = ((w >> 34) == (tag >> 34)) ? uint32_t(w >> 32) & 3u : 0u;
+                v[q] = uint32_t(w);
+            }
         }
-        const uint32_t ready = __ballot_sync(0xffffffffu, flag != 0);
-        const uint32_t inc = __ballot_sync(0xffffffffu, flag == 2);
-        // lanes up to and including the nearest inclusive prefix must be ready
-        const uint32_t need = inc ? (((inc & (0u - inc)) << 1) - 1u) : 0xffffffffu;
-        if ((ready & need) == need) {
-            excl += __reduce_add_sync(0xffffffffu, ((need >> lane) & 1u) ? val : 0u);
-            if (inc) break;
-            j -= 32;
+        int my_inc = kLookbackPerLane;  // this lane's nearest inclusive position
+#pragma unroll
+        for (int q = kLookbackPerLane - 1; q >= 0; --q)
+            if (f[q] == 2) my_inc = q;
+        const uint32_t inc_lanes = __ballot_sync(0xffffffffu, my_inc < kLookbackPerLane);
+        const int L = inc_lanes ? __ffs(inc_lanes) - 1 : 32;
+        const int need = lane < L ? kLookbackPerLane : (lane == L ? my_inc + 1 : 0);
+        bool ready = true;
+        uint32_t sum = 0;
+#pragma unroll
+        for (int q = 0; q < kLookbackPerLane; ++q) {
+            if (q < need) {
+                ready = ready && f[q] != 0;
+                sum += v[q];
+            }
+        }
+        if (__all_sync(0xffffffffu, ready)) {
+            excl += __reduce_add_sync(0xffffffffu, sum);
+            if (L < 32) break;
+            j -= 32 * kLookbackPerLane;
             continue;
         }
-        uint64_t now = __shfl_sync(0xffffffffu, global_ns(), 0);
+        const uint64_t now = __shfl_sync(0xffffffffu, global_ns(), 0);
         if (t0 == 0) {
             t0 = now;
         } else if (now - t0 > kLookbackLimitNs) {
@@ -81,9 +113,9 @@ __device__ uint32_t lookback(unsigned long long *st, uint32_t tile, uint32_t agg
             break;
         }
         __nanosleep(backoff);
-        if (backoff < 1024) backoff <<= 1;
+        if (backoff < 256) backoff <<= 1;
     }
-    if (lane == 0) st_relaxed_u64(st + tile, tag | kFlagInc | (excl + agg));
+    if (lane == 0) st_relaxed_u64(st + chunk, tag | kFlagInc | (excl + agg));
     return excl;
 }
 
@@ -102,15 +134,12 @@ __device__ __forceinline__ bool header_ok(const Header &H, uint64_t n, uint64_t 
     return true;
 }
 
-// Zero [a, b) of out with the whole CTA.
 __device__ __forceinline__ void zero_bytes(uint8_t *out, uint64_t a, uint64_t b) {
     for (uint64_t x = a + threadIdx.x; x < b; x += NT) out[x] = 0;
 }
 
-// Header, offsets[nb] and the zero gaps between sections (done once per stream).
-template <int DT>
-__device__ void write_stream_frame(uint8_t *out, const Layout &L, const uint32_t *hdr, uint64_t n,
-                                   uint64_t E) {
+// Header, offsets[nb] and the zero gaps between sections (once per stream).
+__device__ void write_stream_frame(uint8_t *out, const Layout &L, const uint32_t *hdr, uint64_t E) {
     if (threadIdx.x < 16) reinterpret_cast<uint32_t *>(out)[threadIdx.x] = hdr[threadIdx.x];
     if (threadIdx.x == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * L.nb) = uint32_t(E);
     zero_bytes(out, L.tab_end, L.plane[0]);
@@ -124,216 +153,294 @@ __device__ void write_stream_frame(uint8_t *out, const Layout &L, const uint32_t
     }
 }
 
-// Load up to `valid` elements of 16 bytes starting at byte offset `off` of in.
+// Up to `valid` elements of one lane's 16-byte step at src (byte by byte
+// past the end of the tensor).
 template <int DT>
-__device__ __forceinline__ uint4 load_group(const uint8_t *in, uint64_t off, int valid) {
-    constexpr int kVec = 16 / Dt<DT>::kElemBytes;
-    if (valid >= kVec) return __ldcs(reinterpret_cast<const uint4 *>(in + off));
+__device__ __forceinline__ uint4 load_step(const uint8_t *src, int valid) {
+    if (valid >= Geo<DT>::LE) return __ldcs(reinterpret_cast<const uint4 *>(src));
     uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int j = 0; j < kVec; ++j) {
+    for (int j = 0; j < Geo<DT>::LE; ++j) {
         if (j < valid) {
             if constexpr (DT == SZ_BF16) {
-                const uint32_t b = reinterpret_cast<const uint16_t *>(in + off)[j];
+                const uint32_t b = reinterpret_cast<const uint16_t *>(src)[j];
                 w[j >> 1] |= b << (16 * (j & 1));
             } else {
-                w[j >> 2] |= uint32_t(in[off + j]) << (8 * (j & 3));
+                w[j >> 2] |= uint32_t(src[j]) << (8 * (j & 3));
             }
         }
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Store the low `nbytes` bytes of (lo, hi) at p; full width when nbytes == width.
 __device__ __forceinline__ void store_bytes(uint8_t *p, uint32_t lo, uint32_t hi, int nbytes) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         if (j < nbytes) p[j] = uint8_t(((j < 4) ? lo : hi) >> (8 * (j & 3)));
 }
 
-template <int DT, int MAXB>
-__device__ void encode_tile(const EncodeParams<MAXB> &p, uint32_t job, uint32_t epoch,
-                            TileShared &S) {
-    const int tid = threadIdx.x;
-    const int t = find_tensor<uint32_t, MAXB>(p.tile_begin, p.T, job);
-    const uint32_t tile = job - p.tile_begin[t];
-    const uint64_t n = p.n[t];
-    const uint8_t *in = p.in[t];
-    uint8_t *out = p.out[t];
-    if (tid < 16) S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
+// Per-lane output pointers of one block; each step advances them by a fixed stride.
+struct EPtr {
+    uint8_t *a, *b, *code;  // BF16: sm plane, -, codes ; E5M2: sign, mantissa, codes
+};
 
-    // ---- 1. loads (issued before the header arrives)
-    constexpr int G = (DT == SZ_BF16) ? 2 : 1;          // 16-byte groups per thread
-    constexpr int kGE = (DT == SZ_BF16) ? 8 : 16;       // elements per group
-    const uint64_t e_tile = uint64_t(tile) * kBlock;
-    uint64_t e0[G];
-    int valid[G];
-    uint4 v[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        e0[g] = e_tile + uint64_t(g) * (kBlock / 2) + uint64_t(tid) * kGE;
-        valid[g] = n > e0[g] ? int(min(uint64_t(kGE), n - e0[g])) : 0;
-        v[g] = valid[g] > 0 ? load_group<DT>(in, e0[g] * Dt<DT>::kElemBytes, valid[g])
-                            : make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
-    uint32_t why = 0;
-    if (!header_ok<DT>(H, n, p.cap[t], &why)) {
-        if (tid == 0 && tile == 0) set_error(p.ctl, why, uint32_t(t));
-        return;  // every tile of this tensor takes this branch: no look-back waits on it
-    }
-    // exponent -> code table
-    if (tid < Dt<DT>::kBins) {
-        uint32_t code = kEscape;
-#pragma unroll
-        for (int c = 0; c < int(kCodes); ++c)
-            if (cb_byte(H.cbw, c) == uint32_t(tid)) code = uint32_t(c);
-        S.lut[tid] = uint8_t(code);
-    }
-    __syncthreads();
-    const Layout L = stream_layout(DT, n, H.E);
+template <int DT> struct EStride;
+template <> struct EStride<SZ_BF16> {
+    static constexpr int a = 256, code = 128;
+};
+template <> struct EStride<SZ_FP8_E5M2> {
+    static constexpr int a = 64, b = 128, code = 256;
+};
 
-    // ---- 2. code, split, store
-    uint32_t codes[G][2];   // nibbles of the group's elements (BF16 uses [g][0])
-    uint32_t emask[G];      // escape flags, bit j = element j of the group
+template <int DT>
+__device__ __forceinline__ EPtr block_out(uint8_t *out, const Layout &L, uint64_t e_lane) {
+    EPtr q;
+    q.code = out + L.code + e_lane / 2;
+    if constexpr (DT == SZ_BF16) {
+        q.a = out + L.plane[0] + e_lane;
+        q.b = nullptr;
+    } else {
+        q.a = out + L.plane[0] + e_lane / 8;
+        q.b = out + L.plane[1] + e_lane / 4;
+    }
+    return q;
+}
+
+// Code one lane's step (LE elements in v); when STORE, write its planes and
+// codes.  Returns escape flags: bit 4j for element j.
+template <int DT, bool STORE>
+__device__ __forceinline__ uint64_t code_step(const uint8_t *lut, uint4 v, int valid, const EPtr &q,
+                                              int it) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (DT == SZ_BF16) {
+        uint32_t cw = 0, x[4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const uint32_t w[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
-        if constexpr (DT == SZ_BF16) {
-            uint32_t cw = 0, smp[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t c0 = S.lut[(w[k] >> 7) & 0xFFu];
-                const uint32_t c1 = S.lut[(w[k] >> 23) & 0xFFu];
-                cw |= (c0 | (c1 << 4)) << (8 * k);
-                smp[k] = ((w[k] >> 8) & 0x00800080u) | (w[k] & 0x007F007Fu);
-            }
-            if (valid[g] < 8) cw &= (1u << (4 * valid[g])) - 1u;  // codes past n are 0
-            const uint32_t sm_lo = __byte_perm(smp[0], smp[1], 0x6420);
-            const uint32_t sm_hi = __byte_perm(smp[2], smp[3], 0x6420);
-            codes[g][0] = cw;
-            codes[g][1] = 0;
-            uint32_t m = cw & (cw >> 1) & (cw >> 2) & (cw >> 3) & 0x11111111u;
-            // compress nibble flags (bits 0,4,..,28) into bits 0..7
-            uint32_t bits = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bits |= ((m >> (4 * j)) & 1u) << j;
-            emask[g] = bits;
-            uint8_t *sm_dst = out + L.plane[0] + e0[g];
-            uint8_t *cd_dst = out + L.code + e0[g] / 2;
-            if (valid[g] == 8) {
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t ws = w[k] << 1;  // exponents in bytes 1 and 3
+            const uint32_t c0 = lut[__byte_perm(ws, 0, 0x4441)];
+            const uint32_t c1 = lut[ws >> 24];
+            cw += (c0 << (8 * k)) + (c1 << (8 * k + 4));
+            // bytes 0 and 2: sign<<7 | mantissa of the two elements (bytes 1, 3 unused)
+            x[k] = ((w[k] >> 8) & 0x00800080u) | (w[k] & 0xFF7FFF7Fu);
+        }
+        if (valid < 8) cw &= (1u << (4 * valid)) - 1u;  // codes past n are 0
+        if (STORE) {
+            const uint32_t sm_lo = __byte_perm(x[0], x[1], 0x6420);
+            const uint32_t sm_hi = __byte_perm(x[2], x[3], 0x6420);
+            uint8_t *sm_dst = q.a + it * EStride<DT>::a;
+            uint8_t *cd_dst = q.code + it * EStride<DT>::code;
+            if (valid == 8) {
                 *reinterpret_cast<uint2 *>(sm_dst) = make_uint2(sm_lo, sm_hi);
                 *reinterpret_cast<uint32_t *>(cd_dst) = cw;
-            } else if (valid[g] > 0) {
-                store_bytes(sm_dst, sm_lo, sm_hi, valid[g]);
-                store_bytes(cd_dst, cw, 0, (valid[g] + 1) / 2);
+            } else if (valid > 0) {
+                store_bytes(sm_dst, sm_lo, sm_hi, valid);
+                store_bytes(cd_dst, cw, 0, (valid + 1) / 2);
             }
-        } else {
-            uint32_t cw[2] = {0, 0}, sign = 0, mant = 0;
+        }
+        return escape_nibbles(cw);
+    } else {
+        uint32_t cw[2] = {0, 0}, sign = 0, mant = 0;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 4; ++k) {
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint32_t c = S.lut[(w[k] >> (8 * b + 2)) & 0x1Fu];
-                    cw[k >> 1] |= c << (4 * (4 * (k & 1) + b));
-                }
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t c = lut[(w[k] >> (8 * b + 2)) & 0x1Fu];
+                cw[k >> 1] += c << (4 * (4 * (k & 1) + b));
+            }
+            if (STORE) {
                 sign |= ((((w[k] >> 7) & 0x01010101u) * 0x01020408u) >> 24) << (4 * k);
-                const uint32_t x = w[k] & 0x03030303u;
-                mant |= ((x | (x >> 6) | (x >> 12) | (x >> 18)) & 0xFFu) << (8 * k);
+                mant |= (((w[k] & 0x03030303u) * 0x01041040u) >> 24) << (8 * k);
             }
-            if (valid[g] < 16) {
-                if (valid[g] < 8) {
-                    cw[0] &= (1u << (4 * valid[g])) - 1u;
-                    cw[1] = 0;
-                } else {
-                    cw[1] &= (valid[g] == 8) ? 0u : ((1u << (4 * (valid[g] - 8))) - 1u);
-                }
+        }
+        if (valid < 16) {
+            if (valid < 8) {
+                cw[0] &= (1u << (4 * valid)) - 1u;
+                cw[1] = 0;
+            } else {
+                cw[1] &= (valid == 8) ? 0u : ((1u << (4 * (valid - 8))) - 1u);
             }
-            codes[g][0] = cw[0];
-            codes[g][1] = cw[1];
-            uint32_t bits = 0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t m = cw[h] & (cw[h] >> 1) & (cw[h] >> 2) & (cw[h] >> 3) & 0x11111111u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) bits |= ((m >> (4 * j)) & 1u) << (8 * h + j);
-            }
-            emask[g] = bits;
-            uint8_t *sg_dst = out + L.plane[0] + e0[g] / 8;
-            uint8_t *mt_dst = out + L.plane[1] + e0[g] / 4;
-            uint8_t *cd_dst = out + L.code + e0[g] / 2;
-            if (valid[g] == 16) {
+        }
+        if (STORE) {
+            uint8_t *sg_dst = q.a + it * EStride<DT>::a;
+            uint8_t *mt_dst = q.b + it * EStride<DT>::b;
+            uint8_t *cd_dst = q.code + it * EStride<DT>::code;
+            if (valid == 16) {
                 *reinterpret_cast<uint16_t *>(sg_dst) = uint16_t(sign);
                 *reinterpret_cast<uint32_t *>(mt_dst) = mant;
                 *reinterpret_cast<uint2 *>(cd_dst) = make_uint2(cw[0], cw[1]);
-            } else if (valid[g] > 0) {
-                store_bytes(sg_dst, sign, 0, (valid[g] + 7) / 8);
-                store_bytes(mt_dst, mant, 0, (valid[g] + 3) / 4);
-                store_bytes(cd_dst, cw[0], cw[1], (valid[g] + 1) / 2);
+            } else if (valid > 0) {
+                store_bytes(sg_dst, sign, 0, (valid + 7) / 8);
+                store_bytes(mt_dst, mant, 0, (valid + 3) / 4);
+                store_bytes(cd_dst, cw[0], cw[1], (valid + 1) / 2);
             }
         }
+        return uint64_t(escape_nibbles(cw[0])) | (uint64_t(escape_nibbles(cw[1])) << 32);
     }
+}
 
-    // ---- 3. rank escapes within the tile; stage them in element order
-    uint32_t packed = 0;
-#pragma unroll
-    for (int g = 0; g < G; ++g) packed |= uint32_t(__popc(emask[g])) << (16 * g);
-    uint32_t total_packed;
-    const uint32_t before = block_exclusive_scan<NT>(packed, S.warp, &total_packed);
-    const uint32_t tile_escapes = (total_packed & 0xFFFFu) + (total_packed >> 16);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        uint32_t r = (g == 0) ? (before & 0xFFFFu) : (total_packed & 0xFFFFu) + (before >> 16);
-        uint32_t m = emask[g];
+// Exponent of element j (runtime) of a lane's step.
+template <int DT>
+__device__ __forceinline__ uint32_t exponent_at(uint4 v, uint32_t j) {
+    if constexpr (DT == SZ_BF16) {
+        const uint32_t wj = pick4(v.x, v.y, v.z, v.w, j >> 1);
+        return (wj >> (16 * (j & 1) + 7)) & 0xFFu;
+    } else {
+        const uint32_t wj = pick4(v.x, v.y, v.z, v.w, j >> 2);
+        return (wj >> (8 * (j & 3) + 2)) & 0x1Fu;
+    }
+}
+
+// Rank one step's escapes within the block and hand each to put(rank, exponent).
+template <int DT, typename Put>
+__device__ __forceinline__ void rank_step(uint64_t m, uint4 v, uint32_t &running, Put put) {
+    const uint32_t c = __popcll(m);
+    uint32_t tot;
+    const uint32_t prefix = warp_exclusive_prefix(c, &tot);
+    if (tot) {
+        uint32_t r = running + prefix;
         while (m) {
-            const uint32_t j = __ffs(m) - 1;
+            const uint32_t j = uint32_t(__ffsll(m) - 1) >> 2;  // element, in element order
             m &= m - 1;
-            uint32_t e;
-            if constexpr (DT == SZ_BF16) {
-                const uint32_t wj = pick4(v[g].x, v[g].y, v[g].z, v[g].w, j >> 1);
-                e = (wj >> (16 * (j & 1) + 7)) & 0xFFu;
-            } else {
-                const uint32_t wj = pick4(v[g].x, v[g].y, v[g].z, v[g].w, j >> 2);
-                e = (wj >> (8 * (j & 3) + 2)) & 0x1Fu;
-            }
-            S.esc[r++] = uint8_t(e);
+            put(r++, exponent_at<DT>(v, j));
+        }
+        running += tot;
+    }
+}
+
+// One warp codes block blk of a tensor of n elements: planes and codes go to
+// out; escapes (exponents in element order) go to put(rank, exponent).
+// Returns the block's escape count.
+template <int DT, bool STORE, typename Put>
+__device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t *in, uint64_t n,
+                                               uint64_t blk, const Layout &L, uint8_t *out, Put put) {
+    using G = Geo<DT>;
+    const int lane = threadIdx.x & 31;
+    const uint64_t e_lane = blk * kBlock + uint64_t(lane) * G::LE;
+    const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
+    const EPtr q = block_out<DT>(out, L, e_lane);
+    uint32_t running = 0;
+    if ((blk + 1) * kBlock <= n) {
+        uint4 ring[G::kAhead + 1];
+#pragma unroll
+        for (int i = 0; i < G::kAhead; ++i) ring[i] = __ldcs(reinterpret_cast<const uint4 *>(src + i * 512));
+#pragma unroll
+        for (int it = 0; it < G::IT; ++it) {
+            if (it + G::kAhead < G::IT)
+                ring[(it + G::kAhead) % (G::kAhead + 1)] =
+                    __ldcs(reinterpret_cast<const uint4 *>(src + (it + G::kAhead) * 512));
+            const uint4 v = ring[it % (G::kAhead + 1)];
+            const uint64_t m = code_step<DT, STORE>(lut, v, G::LE, q, it);
+            rank_step<DT>(m, v, running, put);
+        }
+    } else {
+        for (int it = 0; it < G::IT; ++it) {
+            const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
+            const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+            const uint4 v = valid > 0 ? load_step<DT>(src + it * 512, valid) : make_uint4(0, 0, 0, 0);
+            const uint64_t m = code_step<DT, STORE>(lut, v, valid, q, it);
+            rank_step<DT>(m, v, running, put);
         }
     }
+    return running;
+}
 
-    // ---- 4. escape offset of this tile within its tensor
-    if (tid < 32) {
+template <int DT, int MAXB>
+__device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t epoch,
+                             EncShared &S, int &lut_tensor) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
+    const uint32_t chunk = job - p.chunk_begin[t];
+    const uint64_t n = p.n[t];
+    const uint64_t nb = cdiv(n, kBlock);
+    const uint64_t b0 = uint64_t(chunk) * kChunkBlocks;
+    const int nbk = int(min(uint64_t(kChunkBlocks), nb - b0));
+    const uint8_t *in = p.in[t];
+    uint8_t *out = p.out[t];
+
+    if (t != lut_tensor) {
+        if (tid < 16)
+            S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
+        __syncthreads();
+        const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
+        if (tid < Dt<DT>::kBins) {
+            uint32_t code = kEscape;
+#pragma unroll
+            for (int c = 0; c < int(kCodes); ++c)
+                if (cb_byte(H.cbw, c) == uint32_t(tid)) code = uint32_t(c);
+            S.lut[tid] = uint8_t(code);
+        }
+        __syncthreads();
+        lut_tensor = t;
+    }
+    const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
+    uint32_t why = 0;
+    if (!header_ok<DT>(H, n, p.cap[t], &why)) {
+        if (tid == 0 && chunk == 0) set_error(p.ctl, why, uint32_t(t));
+        return;  // every chunk of this tensor takes this branch: no look-back waits on it
+    }
+    const Layout L = stream_layout(DT, n, H.E);
+
+    // ---- each warp codes one block; its escapes are staged in element order
+    uint8_t *stage = S.esc[warp];
+    if (warp < nbk) {
+        const uint32_t cnt = code_block<DT, true>(S.lut, in, n, b0 + warp, L, out,
+                                                  [&](uint32_t r, uint32_t e) {
+                                                      if (r < kWarpStage) stage[r] = uint8_t(e);
+                                                  });
+        if (lane == 0) S.cnt[warp] = cnt;
+    } else if (lane == 0) {
+        S.cnt[warp] = 0;
+    }
+    __syncthreads();
+
+    // ---- block offsets within the chunk, and the chunk's offset in its tensor
+    if (warp == 0) {
+        const uint32_t c = lane < kChunkBlocks ? S.cnt[lane] : 0u;
+        uint32_t x = c;
+#pragma unroll
+        for (int o = 1; o < kChunkBlocks; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, x, kChunkBlocks - 1);
+        if (lane < kChunkBlocks) S.blk_off[lane] = x - c;
         bool timed_out;
-        const uint32_t excl =
-            lookback(p.status + p.tile_begin[t], tile, tile_escapes, epoch, &timed_out);
-        if (tid == 0) {
+        const uint32_t excl = lookback(p.status + p.chunk_begin[t], chunk, total, epoch, &timed_out);
+        if (lane == 0) {
             S.excl = excl;
             if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
+            if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+            if (b0 + nbk == nb && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
         }
     }
     __syncthreads();
     const uint32_t excl = S.excl;
 
-    // ---- 5. escapes, offsets entry, and the stream frame (last tile)
-    const uint64_t dst = L.esc + excl;
-    for (uint32_t x = tid; x < tile_escapes; x += NT)
-        if (dst + x < L.total) out[dst + x] = S.esc[x];
-    if (tid == 0) {
-        *reinterpret_cast<uint32_t *>(out + 64 + 4 * uint64_t(tile)) = excl;
-        if (uint64_t(excl) + tile_escapes > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+    // ---- offsets-table entries and escapes of each block
+    if (warp < nbk) {
+        const uint64_t blk = b0 + warp;
+        const uint32_t cnt = S.cnt[warp];
+        const uint64_t dst = L.esc + excl + S.blk_off[warp];
+        if (lane == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * blk) = excl + S.blk_off[warp];
+        if (cnt <= kWarpStage) {
+            for (uint32_t x = lane; x < cnt; x += 32)
+                if (dst + x < L.total) out[dst + x] = stage[x];
+        } else {
+            // more escapes than the stage holds: re-read the block, write them directly
+            code_block<DT, false>(S.lut, in, n, blk, L, out, [&](uint32_t r, uint32_t e) {
+                if (dst + r < L.total) out[dst + r] = uint8_t(e);
+            });
+        }
     }
-    if (uint64_t(tile) + 1 == L.nb) {
-        if (tid == 0 && uint64_t(excl) + tile_escapes != H.E)
-            set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-        write_stream_frame<DT>(out, L, S.hdr, n, H.E);
-    }
+    if (b0 + nbk == nb) write_stream_frame(out, L, S.hdr, H.E);
 }
 
 // Stream of an empty tensor: header, offsets[0] = 0, zero padding.
 template <int DT, int MAXB>
-__device__ void encode_empty(const EncodeParams<MAXB> &p, int t, TileShared &S) {
+__device__ void encode_empty(const EncodeParams<MAXB> &p, int t, EncShared &S) {
     const int tid = threadIdx.x;
-    if (tid < 16) S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
+    if (tid < 16)
+        S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
     __syncthreads();
     const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
     uint32_t why = 0;
@@ -341,27 +448,34 @@ __device__ void encode_empty(const EncodeParams<MAXB> &p, int t, TileShared &S) 
         if (tid == 0) set_error(p.ctl, why, uint32_t(t));
         return;
     }
-    const Layout L = stream_layout(DT, 0, 0);
-    write_stream_frame<DT>(p.out[t], L, S.hdr, 0, 0);
+    write_stream_frame(p.out[t], stream_layout(DT, 0, 0), S.hdr, 0);
 }
 
 template <int DT, int MAXB>
 __global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
-    __shared__ TileShared S;
-    __shared__ uint32_t s_job, s_epoch;
+    __shared__ EncShared S;
     const int tid = threadIdx.x;
     if (tid == 0) {
-        s_job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
-        s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
+        S.job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
+        S.excl = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
     }
     __syncthreads();
-    const uint32_t job = s_job, epoch = s_epoch;
-    if (job < p.total_tiles)
-        encode_tile<DT, MAXB>(p, job, epoch, S);
-    else if (job < p.total_jobs)
-        encode_empty<DT, MAXB>(p, p.empty[job - p.total_tiles], S);
+    const uint32_t epoch = S.excl;
+    uint32_t job = S.job;
+    int lut_tensor = -1;
+    while (job < p.total_jobs) {
+        if (job < p.total_chunks) {
+            encode_chunk<DT, MAXB>(p, job, epoch, S, lut_tensor);
+        } else {
+            encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], S);
+            lut_tensor = -1;
+        }
+        __syncthreads();
+        if (tid == 0) S.job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
+        __syncthreads();
+        job = S.job;
+    }
     // The last CTA to retire leaves the counters ready for the next launch.
-    __syncthreads();
     if (tid == 0) {
         __threadfence();
         if (atomicAdd(&p.ctl[kCtlDone], 1u) == gridDim.x - 1) {
@@ -374,25 +488,33 @@ __global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ Enco
 
 template <int DT, int MAXB>
 sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
+    auto kern = encode_kernel<DT, MAXB>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, 0) != cudaSuccess || per_sm < 1)
+        return SZ_ERR_CUDA;
+    const uint64_t resident = uint64_t(a.num_sms) * per_sm;
     EncodeParams<MAXB> p;
     p.ctl = a.ctl;
     p.status = a.status;
     p.plans = a.plans;
     p.T = a.T;
     p.n_empty = 0;
-    p.tile_begin[0] = 0;
+    p.chunk_log2 = 3;  // one block per warp
+    p.chunk_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
         p.in[t] = static_cast<const uint8_t *>(a.in[t]);
         p.out[t] = static_cast<uint8_t *>(a.out[t]);
         p.n[t] = a.n[t];
         p.cap[t] = a.cap[t];
-        p.tile_begin[t + 1] = p.tile_begin[t] + uint32_t(cdiv(a.n[t], kBlock));
+        const uint64_t nb = cdiv(a.n[t], kBlock);
+        p.chunk_begin[t + 1] = p.chunk_begin[t] + uint32_t(cdiv(nb, uint64_t(kChunkBlocks)));
         if (a.n[t] == 0) p.empty[p.n_empty++] = uint16_t(t);
     }
-    p.total_tiles = p.tile_begin[a.T];
-    p.total_jobs = p.total_tiles + uint32_t(p.n_empty);
+    p.total_chunks = p.chunk_begin[a.T];
+    p.total_jobs = p.total_chunks + uint32_t(p.n_empty);
     if (p.total_jobs == 0) return SZ_OK;
-    encode_kernel<DT, MAXB><<<p.total_jobs, NT, 0, stream>>>(p);
+    const uint64_t grid = p.total_jobs < resident ? p.total_jobs : resident;
+    kern<<<unsigned(grid), NT, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
 

@@ -6,15 +6,18 @@
 // (count descending, value ascending), takes the first 15 as the codebook and
 // writes the 64-byte plan (= stream header: n, E, codebook, total bytes).
 //
-// Histogram design (B200): each thread owns a private column of packed 16-bit
-// counters in shared memory (word r of thread t at s_cols[r * NT + t] holds
-// the counts of exponent values 2r and 2r+1).  Lane t of every warp always
-// touches bank t % 32, so the shared-memory atomics never conflict and never
-// contend, whatever the exponent distribution (an all-zero tensor costs the
-// same as a spread one).  Counters are flushed to the tensor's global
-// histogram (one atomic per non-zero bin per CTA) before any thread can have
-// counted 65535 elements.  Input is streamed with 16-byte read-only loads, a
-// software-pipelined batch of U vectors per thread in flight.
+// Histogram design (B200): counters live in shared memory as 16-bit halves of
+// 32-bit words.  Word (e, c) at s_cols[e * NT/2 + c] holds two counts of
+// exponent value e: the low half belongs to thread c, the high half to thread
+// c + NT/2.  A thread therefore adds a constant (1 or 1 << 16) to one word per
+// element: a shift, a mask and one shared-memory atomic.  Lane l of any warp
+// always hits bank l % 32 and no two lanes of a warp share a word, so the
+// atomics never conflict and never contend, whatever the exponent
+// distribution (an all-zero tensor costs the same as a spread one).  Counters
+// are flushed to the tensor's global histogram (one atomic per non-zero bin
+// per CTA) before any thread can have counted 65535 elements.  Input is
+// streamed with 16-byte read-only loads, a software-pipelined batch of U
+// vectors per thread in flight.
 #include "sz_common.cuh"
 #include "sz_internal.h"
 
@@ -23,37 +26,34 @@ namespace sz {
 namespace {
 
 constexpr int kPlanThreads = 256;
-constexpr int kPlanUnroll = 8;                // 16-byte vectors in flight per thread
+constexpr int kPlanUnroll = 12;               // 16-byte vectors in flight per thread
 constexpr uint32_t kItemBytes = 16384;        // partition unit of the input
 constexpr uint32_t kMaxPerThread = 65535;     // 16-bit counter limit
 
 template <int DT>
 struct PlanCfg {
     static constexpr int kBins = Dt<DT>::kBins;
-    static constexpr int kRows = kBins / 2;                 // packed counter words per thread
     static constexpr int kElemBytes = Dt<DT>::kElemBytes;
     static constexpr int kVecElems = 16 / kElemBytes;       // elements per 16-byte vector
     static constexpr uint32_t kItemElems = kItemBytes / kElemBytes;
 };
 
-// Count the elements of one 16-byte vector into this thread's column.
+// Count the elements of one 16-byte vector.  col = this thread's column
+// (s_cols + tid % (NT/2)); inc = its half (1 or 1 << 16).
 template <int DT, int NT>
-__device__ __forceinline__ void count_vec(uint32_t *col, uint4 v) {
+__device__ __forceinline__ void count_vec(uint32_t *col, uint32_t inc, uint4 v) {
+    constexpr int kRow = NT / 2;  // words per exponent value
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         if constexpr (DT == SZ_BF16) {
             // two elements per word: exponent bits 7..14 and 23..30
-            const uint32_t e0 = (w[k] >> 7) & 0xFFu, e1 = (w[k] >> 23) & 0xFFu;
-            atomicAdd(col + (e0 >> 1) * NT, 1u << ((e0 & 1u) << 4));
-            atomicAdd(col + (e1 >> 1) * NT, 1u << ((e1 & 1u) << 4));
+            atomicAdd(col + ((w[k] >> 7) & 0xFFu) * kRow, inc);
+            atomicAdd(col + ((w[k] >> 23) & 0xFFu) * kRow, inc);
         } else {
             // four elements per word: exponent bits 2..6 of each byte
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t e = (w[k] >> (8 * b + 2)) & 0x1Fu;
-                atomicAdd(col + (e >> 1) * NT, 1u << ((e & 1u) << 4));
-            }
+            for (int b = 0; b < 4; ++b) atomicAdd(col + ((w[k] >> (8 * b + 2)) & 0x1Fu) * kRow, inc);
         }
     }
 }
@@ -70,7 +70,7 @@ __device__ __forceinline__ uint32_t exponent_scalar(const uint8_t *in, uint64_t 
 
 // Count elements [a, b) of one tensor (a is a multiple of the vector size).
 template <int DT, int NT>
-__device__ void count_range(uint32_t *col, const uint8_t *in, uint64_t a, uint64_t b) {
+__device__ void count_range(uint32_t *col, uint32_t inc, const uint8_t *in, uint64_t a, uint64_t b) {
     using C = PlanCfg<DT>;
     constexpr int U = kPlanUnroll;
     const uint4 *src = reinterpret_cast<const uint4 *>(in) + a / C::kVecElems;
@@ -93,41 +93,35 @@ __device__ void count_range(uint32_t *col, const uint8_t *in, uint64_t a, uint64
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const uint64_t k = base + tid + uint64_t(u) * NT;
-            if (k < nvec) count_vec<DT, NT>(col, cur[u]);
+            if (k < nvec) count_vec<DT, NT>(col, inc, cur[u]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) cur[u] = nxt[u];
     }
     // ragged end (< one vector): thread 0 counts it element by element
     if (tid == 0) {
-        for (uint64_t i = a + nvec * C::kVecElems; i < b; ++i) {
-            const uint32_t e = exponent_scalar<DT>(in, i);
-            atomicAdd(col + (e >> 1) * NT, 1u << ((e & 1u) << 4));
-        }
+        for (uint64_t i = a + nvec * C::kVecElems; i < b; ++i)
+            atomicAdd(col + exponent_scalar<DT>(in, i) * (NT / 2), inc);
     }
 }
 
-// Add every thread's column into the global histogram g_hist and clear them.
+// Add every column into the global histogram g_hist and clear them.
 template <int DT, int NT>
 __device__ void flush_columns(uint32_t *s_cols, uint32_t *g_hist) {
     using C = PlanCfg<DT>;
+    constexpr int kRow = NT / 2;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     __syncthreads();
-    for (int r = warp; r < C::kRows; r += NT / 32) {
-        uint32_t lo = 0, hi = 0;
+    for (int e = warp; e < C::kBins; e += NT / 32) {
+        uint32_t sum = 0;
 #pragma unroll
-        for (int c = lane; c < NT; c += 32) {
-            const uint32_t w = s_cols[r * NT + c];
-            s_cols[r * NT + c] = 0;
-            lo += w & 0xFFFFu;
-            hi += w >> 16;
+        for (int c = lane; c < kRow; c += 32) {
+            const uint32_t w = s_cols[e * kRow + c];
+            s_cols[e * kRow + c] = 0;
+            sum += (w & 0xFFFFu) + (w >> 16);
         }
-        lo = __reduce_add_sync(0xffffffffu, lo);
-        hi = __reduce_add_sync(0xffffffffu, hi);
-        if (lane == 0) {
-            if (lo) atomicAdd(g_hist + 2 * r, lo);
-            if (hi) atomicAdd(g_hist + 2 * r + 1, hi);
-        }
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0 && sum) atomicAdd(g_hist + e, sum);
     }
     __threadfence();
     __syncthreads();
@@ -196,13 +190,14 @@ __device__ void select_codebook(uint32_t *g_hist, uint32_t *g_ticket, uint64_t n
 template <int DT, int NT, int MAXB>
 __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ PlanParams<MAXB> p) {
     using C = PlanCfg<DT>;
-    extern __shared__ uint32_t s_cols[];  // C::kRows * NT packed counters
+    extern __shared__ uint32_t s_cols[];  // C::kBins * NT/2 words of two 16-bit counters
     __shared__ uint32_t s_cnt[C::kBins];
     __shared__ uint8_t s_cb[16];
     __shared__ uint32_t s_words[16];
     __shared__ uint32_t s_last;
     const int tid = threadIdx.x;
-    uint32_t *col = s_cols + tid;
+    uint32_t *col = s_cols + (tid % (NT / 2));
+    const uint32_t inc = 1u << (16 * (tid / (NT / 2)));
 
     // Plans of empty tensors: codebook of the 15 smallest values, E = 0.
     if (blockIdx.x == 0) {
@@ -222,7 +217,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
     const uint64_t lo = p.total_items * blockIdx.x / gridDim.x;
     const uint64_t hi = p.total_items * (blockIdx.x + 1) / gridDim.x;
     if (lo >= hi) return;
-    for (int r = 0; r < C::kRows; ++r) s_cols[r * NT + tid] = 0;
+    for (int i = tid; i < C::kBins * (NT / 2); i += NT) s_cols[i] = 0;
     __syncthreads();
 
     int t = find_tensor<uint64_t, MAXB>(p.item_begin, p.T, lo);
@@ -236,7 +231,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
         // sub-ranges short enough that no 16-bit counter can overflow
         constexpr uint64_t kSub = uint64_t(kMaxPerThread / C::kVecElems) * C::kVecElems * NT;
         for (uint64_t s = a; s < b; s += kSub) {
-            count_range<DT, NT>(col, p.in[t], s, min(b, s + kSub));
+            count_range<DT, NT>(col, inc, p.in[t], s, min(b, s + kSub));
             flush_columns<DT, NT>(s_cols, g_hist);
         }
         // ticket: the CTA that completes the tensor's last item selects its codebook
@@ -274,7 +269,7 @@ sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
         p.item_begin[t + 1] = p.item_begin[t] + cdiv(a.n[t], C::kItemElems);
     }
     p.total_items = p.item_begin[a.T];
-    const size_t smem = size_t(C::kRows) * NT * 4;
+    const size_t smem = size_t(C::kBins) * (NT / 2) * 4;
     auto kern = plan_kernel<DT, NT, MAXB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
         cudaSuccess)

@@ -154,9 +154,10 @@ def test_lookback_wait_times_out_and_reports():
     SZ_ERR_TIMEOUT, the kernel returns, and the context stays usable.
 
     The workspace's job counter (control word 3) is moved to 1 on the host, so job 0
-    -- tile 0 of the tensor -- is never run and its status word is never set."""
+    -- the tensor's first chunk of blocks -- is never run and its status word is
+    never set; every later chunk's look-back waits on it."""
     m = sz()
-    n = 4096 * 8
+    n = 4096 * 64
     x = kvgen.stress_tensor(n, 10, 77).cuda()
     ws = m.new_workspace(0, [n])
     plan = m.new_plans(1)
