@@ -19,6 +19,8 @@
 //     escape bytes from a shuffle; the elements are reassembled with byte
 //     permutes and integer multiply-adds and written with 16-byte stores
 //     (512 contiguous bytes per warp instruction).
+#include <type_traits>
+
 #include "sz_common.cuh"
 #include "sz_internal.h"
 
@@ -233,7 +235,8 @@ __device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab,
                                             int valid, uint32_t &running, uint32_t esc_reg,
                                             const uint8_t *esc_g, uint32_t cnt, bool &bad) {
     uint32_t o[4];
-    uint64_t m;  // escape flags of this lane's elements: bit 4j for element j
+    // escape flags of this lane's elements: bit 4j for element j
+    typename std::conditional<DT == SZ_BF16, uint32_t, uint64_t>::type m;
     if constexpr (DT == SZ_BF16) {
         const uint32_t cw = f.c0;
 #pragma unroll
@@ -258,17 +261,18 @@ __device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab,
         }
         m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
     }
-    const uint32_t c = __popcll(m);
+    const uint32_t c = (DT == SZ_BF16) ? uint32_t(__popc(uint32_t(m))) : uint32_t(__popcll(uint64_t(m)));
     uint32_t tot;
     const uint32_t prefix = warp_exclusive_prefix(c, &tot);
     if (tot) {
         const uint32_t maxc = __reduce_max_sync(0xffffffffu, c);
-        uint64_t mm = m;
+        auto mm = m;
         for (uint32_t i = 0; i < maxc; ++i) {
             const uint32_t r = running + prefix + i;
             const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
             if (i < c) {
-                const uint32_t j = uint32_t(__ffsll(mm) - 1) >> 2;  // element, in element order
+                // element, in element order
+                const uint32_t j = uint32_t((DT == SZ_BF16) ? __ffs(uint32_t(mm)) - 1 : __ffsll(uint64_t(mm)) - 1) >> 2;
                 mm &= mm - 1;
                 uint32_t e = 0;
                 if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);

@@ -27,20 +27,20 @@ namespace {
 
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
-constexpr int kChunkBlocks = NW;                      // a chunk is one block per warp
-constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per block
+constexpr int kChunkBlocks = 4;                       // a warp's unit of work: 4 consecutive blocks
+constexpr uint32_t kWarpStage = 4096;                 // staged escape bytes per chunk
 constexpr int kLookbackPerLane = 4;                   // status words per lane per step
 constexpr uint64_t kLookbackLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate published
 constexpr unsigned long long kFlagInc = 2ull << 32;   // inclusive prefix published
 
-struct EncShared {
+// Each warp works alone: its own plan header, exponent -> code table and
+// escape stage.
+struct alignas(16) WarpShared {
     uint32_t hdr[16];
-    uint32_t cnt[kChunkBlocks];      // escapes of each block of the chunk
     uint32_t blk_off[kChunkBlocks];  // escapes before each block, within the chunk
-    uint32_t job, excl;
-    uint8_t lut[256];                // exponent -> code
-    alignas(16) uint8_t esc[kChunkBlocks][kWarpStage];
+    uint8_t lut[256];
+    uint8_t esc[kWarpStage];
 };
 
 template <int DT>
@@ -50,7 +50,7 @@ struct Geo {
     static constexpr int kAhead = 3;                        // steps of loads in flight
 };
 
-// Decoupled look-back, run by warp 0.  Returns the escapes in the tensor's
+// Decoupled look-back, run by one warp.  Returns the escapes in the tensor's
 // chunks before `chunk`; publishes this chunk's aggregate at once and its
 // inclusive prefix when known.  Status word: epoch (30 bits) << 34 |
 // flag << 32 | value; words of earlier launches carry an older epoch and read
@@ -135,13 +135,14 @@ __device__ __forceinline__ bool header_ok(const Header &H, uint64_t n, uint64_t 
 }
 
 __device__ __forceinline__ void zero_bytes(uint8_t *out, uint64_t a, uint64_t b) {
-    for (uint64_t x = a + threadIdx.x; x < b; x += NT) out[x] = 0;
+    for (uint64_t x = a + (threadIdx.x & 31); x < b; x += 32) out[x] = 0;
 }
 
-// Header, offsets[nb] and the zero gaps between sections (once per stream).
+// Header, offsets[nb] and the zero gaps between sections (once per stream, one warp).
 __device__ void write_stream_frame(uint8_t *out, const Layout &L, const uint32_t *hdr, uint64_t E) {
-    if (threadIdx.x < 16) reinterpret_cast<uint32_t *>(out)[threadIdx.x] = hdr[threadIdx.x];
-    if (threadIdx.x == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * L.nb) = uint32_t(E);
+    const int lane = threadIdx.x & 31;
+    if (lane < 16) reinterpret_cast<uint32_t *>(out)[lane] = hdr[lane];
+    if (lane == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * L.nb) = uint32_t(E);
     zero_bytes(out, L.tab_end, L.plane[0]);
 #pragma unroll
     for (int s = 0; s < 3; ++s) {
@@ -344,10 +345,30 @@ __device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t
     return running;
 }
 
+// Load tensor t's plan into the warp's shared area and build its exponent ->
+// code table.
+template <int DT, int MAXB>
+__device__ __forceinline__ void warp_load_plan(const EncodeParams<MAXB> &p, int t, WarpShared &W) {
+    const int lane = threadIdx.x & 31;
+    if (lane < 16)
+        W.hdr[lane] = lane < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[lane] : 0u;
+    __syncwarp();
+    const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
+    for (int e = lane; e < Dt<DT>::kBins; e += 32) {
+        uint32_t code = kEscape;
+#pragma unroll
+        for (int c = 0; c < int(kCodes); ++c)
+            if (cb_byte(H.cbw, c) == uint32_t(e)) code = uint32_t(c);
+        W.lut[e] = uint8_t(code);
+    }
+    __syncwarp();
+}
+
+// One warp encodes chunk `chunk` (up to 4 blocks) of tensor t.
 template <int DT, int MAXB>
 __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t epoch,
-                             EncShared &S, int &lut_tensor) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+                             WarpShared &W, int &plan_tensor) {
+    const int lane = threadIdx.x & 31;
     const int t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
     const uint32_t chunk = job - p.chunk_begin[t];
     const uint64_t n = p.n[t];
@@ -357,125 +378,98 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
     const uint8_t *in = p.in[t];
     uint8_t *out = p.out[t];
 
-    if (t != lut_tensor) {
-        if (tid < 16)
-            S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
-        __syncthreads();
-        const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
-        if (tid < Dt<DT>::kBins) {
-            uint32_t code = kEscape;
-#pragma unroll
-            for (int c = 0; c < int(kCodes); ++c)
-                if (cb_byte(H.cbw, c) == uint32_t(tid)) code = uint32_t(c);
-            S.lut[tid] = uint8_t(code);
-        }
-        __syncthreads();
-        lut_tensor = t;
+    if (t != plan_tensor) {
+        warp_load_plan<DT, MAXB>(p, t, W);
+        plan_tensor = t;
     }
-    const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
+    const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     uint32_t why = 0;
     if (!header_ok<DT>(H, n, p.cap[t], &why)) {
-        if (tid == 0 && chunk == 0) set_error(p.ctl, why, uint32_t(t));
+        if (lane == 0 && chunk == 0) set_error(p.ctl, why, uint32_t(t));
         return;  // every chunk of this tensor takes this branch: no look-back waits on it
     }
     const Layout L = stream_layout(DT, n, H.E);
 
-    // ---- each warp codes one block; its escapes are staged in element order
-    uint8_t *stage = S.esc[warp];
-    if (warp < nbk) {
-        const uint32_t cnt = code_block<DT, true>(S.lut, in, n, b0 + warp, L, out,
-                                                  [&](uint32_t r, uint32_t e) {
-                                                      if (r < kWarpStage) stage[r] = uint8_t(e);
-                                                  });
-        if (lane == 0) S.cnt[warp] = cnt;
-    } else if (lane == 0) {
-        S.cnt[warp] = 0;
+    // ---- code the chunk's blocks; stage escapes in element order
+    uint32_t running = 0;
+#pragma unroll 1
+    for (int k = 0; k < nbk; ++k) {
+        if (lane == 0) W.blk_off[k] = running;
+        const uint32_t base = running;
+        running += code_block<DT, true>(W.lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+            if (base + r < kWarpStage) W.esc[base + r] = uint8_t(e);
+        });
     }
-    __syncthreads();
+    __syncwarp();
 
-    // ---- block offsets within the chunk, and the chunk's offset in its tensor
-    if (warp == 0) {
-        const uint32_t c = lane < kChunkBlocks ? S.cnt[lane] : 0u;
-        uint32_t x = c;
-#pragma unroll
-        for (int o = 1; o < kChunkBlocks; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        const uint32_t total = __shfl_sync(0xffffffffu, x, kChunkBlocks - 1);
-        if (lane < kChunkBlocks) S.blk_off[lane] = x - c;
-        bool timed_out;
-        const uint32_t excl = lookback(p.status + p.chunk_begin[t], chunk, total, epoch, &timed_out);
-        if (lane == 0) {
-            S.excl = excl;
-            if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
-            if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-            if (b0 + nbk == nb && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-        }
+    // ---- escape offset of the chunk within its tensor
+    bool timed_out;
+    const uint32_t excl = lookback(p.status + p.chunk_begin[t], chunk, running, epoch, &timed_out);
+    if (lane == 0) {
+        if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
+        if (uint64_t(excl) + running > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+        if (b0 + nbk == nb && uint64_t(excl) + running != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
     }
-    __syncthreads();
-    const uint32_t excl = S.excl;
 
-    // ---- offsets-table entries and escapes of each block
-    if (warp < nbk) {
-        const uint64_t blk = b0 + warp;
-        const uint32_t cnt = S.cnt[warp];
-        const uint64_t dst = L.esc + excl + S.blk_off[warp];
-        if (lane == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * blk) = excl + S.blk_off[warp];
-        if (cnt <= kWarpStage) {
-            for (uint32_t x = lane; x < cnt; x += 32)
-                if (dst + x < L.total) out[dst + x] = stage[x];
-        } else {
-            // more escapes than the stage holds: re-read the block, write them directly
-            code_block<DT, false>(S.lut, in, n, blk, L, out, [&](uint32_t r, uint32_t e) {
-                if (dst + r < L.total) out[dst + r] = uint8_t(e);
+    // ---- offsets-table entries and escapes
+    if (lane < nbk) *reinterpret_cast<uint32_t *>(out + 64 + 4 * (b0 + lane)) = excl + W.blk_off[lane];
+    const uint64_t dst = L.esc + excl;
+    if (running <= kWarpStage) {
+        __syncwarp();
+        for (uint32_t x = lane; x < running; x += 32)
+            if (dst + x < L.total) out[dst + x] = W.esc[x];
+    } else {
+        // more escapes than the stage holds: re-read the chunk, write them directly
+#pragma unroll 1
+        for (int k = 0; k < nbk; ++k) {
+            const uint64_t d = dst + W.blk_off[k];
+            code_block<DT, false>(W.lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+                if (d + r < L.total) out[d + r] = uint8_t(e);
             });
         }
     }
-    if (b0 + nbk == nb) write_stream_frame(out, L, S.hdr, H.E);
+    if (b0 + nbk == nb) write_stream_frame(out, L, W.hdr, H.E);
+    __syncwarp();  // the stage may be refilled by the next chunk
 }
 
-// Stream of an empty tensor: header, offsets[0] = 0, zero padding.
+// Stream of an empty tensor: header, offsets[0] = 0, zero padding (one warp).
 template <int DT, int MAXB>
-__device__ void encode_empty(const EncodeParams<MAXB> &p, int t, EncShared &S) {
-    const int tid = threadIdx.x;
-    if (tid < 16)
-        S.hdr[tid] = tid < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[tid] : 0u;
-    __syncthreads();
-    const Header H = load_header(reinterpret_cast<const uint8_t *>(S.hdr));
+__device__ void encode_empty(const EncodeParams<MAXB> &p, int t, WarpShared &W, int &plan_tensor) {
+    const int lane = threadIdx.x & 31;
+    warp_load_plan<DT, MAXB>(p, t, W);
+    plan_tensor = t;
+    const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     uint32_t why = 0;
     if (!header_ok<DT>(H, 0, p.cap[t], &why)) {
-        if (tid == 0) set_error(p.ctl, why, uint32_t(t));
+        if (lane == 0) set_error(p.ctl, why, uint32_t(t));
         return;
     }
-    write_stream_frame(p.out[t], stream_layout(DT, 0, 0), S.hdr, 0);
+    write_stream_frame(p.out[t], stream_layout(DT, 0, 0), W.hdr, 0);
 }
 
 template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
-    __shared__ EncShared S;
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        S.job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
-        S.excl = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
-    }
+__global__ void __launch_bounds__(NT, 4) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
+    __shared__ WarpShared s_warp[NW];
+    __shared__ uint32_t s_epoch;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
     __syncthreads();
-    const uint32_t epoch = S.excl;
-    uint32_t job = S.job;
-    int lut_tensor = -1;
-    while (job < p.total_jobs) {
-        if (job < p.total_chunks) {
-            encode_chunk<DT, MAXB>(p, job, epoch, S, lut_tensor);
-        } else {
-            encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], S);
-            lut_tensor = -1;
-        }
-        __syncthreads();
-        if (tid == 0) S.job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
-        __syncthreads();
-        job = S.job;
+    const uint32_t epoch = s_epoch;
+    WarpShared &W = s_warp[warp];
+    int plan_tensor = -1;
+    // every warp claims chunks in launch order until none is left
+    while (true) {
+        uint32_t job = 0;
+        if (lane == 0) job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
+        job = __shfl_sync(0xffffffffu, job, 0);
+        if (job >= p.total_jobs) break;
+        if (job < p.total_chunks)
+            encode_chunk<DT, MAXB>(p, job, epoch, W, plan_tensor);
+        else
+            encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], W, plan_tensor);
     }
     // The last CTA to retire leaves the counters ready for the next launch.
+    __syncthreads();
     if (tid == 0) {
         __threadfence();
         if (atomicAdd(&p.ctl[kCtlDone], 1u) == gridDim.x - 1) {
@@ -499,7 +493,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     p.plans = a.plans;
     p.T = a.T;
     p.n_empty = 0;
-    p.chunk_log2 = 3;  // one block per warp
+    p.chunk_log2 = 2;  // kChunkBlocks
     p.chunk_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
         p.in[t] = static_cast<const uint8_t *>(a.in[t]);
@@ -513,7 +507,8 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     p.total_chunks = p.chunk_begin[a.T];
     p.total_jobs = p.total_chunks + uint32_t(p.n_empty);
     if (p.total_jobs == 0) return SZ_OK;
-    const uint64_t grid = p.total_jobs < resident ? p.total_jobs : resident;
+    const uint64_t need = cdiv(p.total_jobs, NW);
+    const uint64_t grid = need < resident ? need : resident;
     kern<<<unsigned(grid), NT, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
