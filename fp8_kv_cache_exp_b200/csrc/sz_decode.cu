@@ -68,23 +68,23 @@ struct WarpStream {
     uint64_t code, pa, pb, esc;   // section offsets in the stream
 };
 
-// Step `it` (within a quarter block) from a shared-memory stage.
+// Step `it` (within a quarter block) from the shared-memory stage at address st.
 template <int DT>
-__device__ __forceinline__ DFrag read_stage(const uint8_t *st, int it) {
-    const int lane = threadIdx.x & 31;
+__device__ __forceinline__ DFrag read_stage(uint32_t st, int it) {
+    const uint32_t lane = threadIdx.x & 31;
     DFrag f;
     if constexpr (DT == SZ_BF16) {
-        f.c0 = *reinterpret_cast<const uint32_t *>(st + it * 128 + lane * 4);
+        f.c0 = lds_u32(st + it * 128 + lane * 4);
         f.c1 = 0;
-        const uint2 s = *reinterpret_cast<const uint2 *>(st + DGeo<DT>::kA + it * 256 + lane * 8);
+        const uint2 s = lds_u64(st + DGeo<DT>::kA + it * 256 + lane * 8);
         f.a = s.x;
         f.b = s.y;
     } else {
-        const uint2 c = *reinterpret_cast<const uint2 *>(st + it * 256 + lane * 8);
+        const uint2 c = lds_u64(st + it * 256 + lane * 8);
         f.c0 = c.x;
         f.c1 = c.y;
-        f.a = *reinterpret_cast<const uint16_t *>(st + DGeo<DT>::kA + it * 64 + lane * 2);
-        f.b = *reinterpret_cast<const uint32_t *>(st + DGeo<DT>::kB + it * 128 + lane * 4);
+        f.a = lds_u16(st + DGeo<DT>::kA + it * 64 + lane * 2);
+        f.b = lds_u32(st + DGeo<DT>::kB + it * 128 + lane * 4);
     }
     return f;
 }
@@ -231,7 +231,7 @@ __device__ __forceinline__ void patch(uint32_t (&o)[4], uint32_t j, uint32_t e) 
 // esc_reg: lane i holds the block's escape i (i < 32); esc_g: the block's
 // escapes in global memory; cnt: escapes the offsets table gives the block.
 template <int DT, bool PARTIAL>
-__device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab, uint8_t *dst,
+__device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, uint8_t *dst,
                                             int valid, uint32_t &running, uint32_t esc_reg,
                                             const uint8_t *esc_g, uint32_t cnt, bool &bad) {
     uint32_t o[4];
@@ -241,7 +241,7 @@ __device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab,
         const uint32_t cw = f.c0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const uint32_t e2 = tab[(cw >> (8 * k)) & 0xFFu];
+            const uint32_t e2 = lds_u32(tab + (((cw >> (8 * k)) & 0xFFu) << 2));
             const uint32_t x = __byte_perm((k < 2) ? f.a : f.b, 0, (k & 1) ? 0x4342 : 0x4140);
             o[k] = x + (x & 0x00800080u) * 0xFFu + (e2 << 7);
         }
@@ -250,8 +250,8 @@ __device__ __forceinline__ void decode_step(const DFrag &f, const uint32_t *tab,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const uint32_t cw = (k < 2) ? f.c0 : f.c1;
-            const uint32_t lo = tab[(cw >> (16 * (k & 1))) & 0xFFu];
-            const uint32_t hi = tab[(cw >> (16 * (k & 1) + 8)) & 0xFFu];
+            const uint32_t lo = lds_u32(tab + (((cw >> (16 * (k & 1))) & 0xFFu) << 2));
+            const uint32_t hi = lds_u32(tab + (((cw >> (16 * (k & 1) + 8)) & 0xFFu) << 2));
             const uint32_t e4 = lo | (hi << 16);
             const uint32_t s4 = (f.a >> (4 * k)) & 0xFu;
             const uint32_t sgn = (s4 * 0x10204080u) & 0x80808080u;
@@ -367,6 +367,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
     extern __shared__ __align__(128) uint8_t s_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpSmem &W = reinterpret_cast<WarpSmem *>(s_raw)[warp];
+    const uint32_t tab_addr = smem_u32(W.tab);
     if (lane == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&W.bar[i], 1);
         fence_mbar_init();
@@ -419,10 +420,11 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
             if (q == 1 && next_same && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
             if (ok && !timed_out) {
                 if (full) {
+                    const uint32_t st_addr = smem_u32(W.stage[st]);
 #pragma unroll
                     for (int it = 0; it < G::QIT; ++it) {
-                        const DFrag f = read_stage<DT>(W.stage[st], it);
-                        decode_step<DT, false>(f, W.tab, out + (q * G::QIT + it) * 512, G::LE, running,
+                        const DFrag f = read_stage<DT>(st_addr, it);
+                        decode_step<DT, false>(f, tab_addr, out + (q * G::QIT + it) * 512, G::LE, running,
                                                esc_reg, esc_g, cnt, bad);
                     }
                 } else {
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
                         const int64_t left = int64_t(ws.n) - e;
                         const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
                         const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
-                        decode_step<DT, true>(f, W.tab, out + it * 512, valid, running, esc_reg, esc_g, cnt, bad);
+                        decode_step<DT, true>(f, tab_addr, out + it * 512, valid, running, esc_reg, esc_g, cnt, bad);
                     }
                 }
             }

@@ -18,6 +18,8 @@
 //      contiguously (a chunk whose escapes overflow the stage re-reads its
 //      input and writes them directly); the tensor's last chunk also writes
 //      the header, offsets[nb] and the zero padding between sections.
+#include <type_traits>
+
 #include "sz_common.cuh"
 #include "sz_internal.h"
 
@@ -207,10 +209,20 @@ __device__ __forceinline__ EPtr block_out(uint8_t *out, const Layout &L, uint64_
     return q;
 }
 
+// Escape flags of one lane's step: bit 4j for element j (32 bits hold BF16's 8
+// elements, 64 bits E5M2's 16).
+template <int DT>
+using EMask = typename std::conditional<DT == SZ_BF16, uint32_t, uint64_t>::type;
+
+__device__ __forceinline__ uint32_t popc_mask(uint32_t m) { return __popc(m); }
+__device__ __forceinline__ uint32_t popc_mask(uint64_t m) { return __popcll(m); }
+__device__ __forceinline__ uint32_t first_bit(uint32_t m) { return __ffs(m) - 1; }
+__device__ __forceinline__ uint32_t first_bit(uint64_t m) { return __ffsll(m) - 1; }
+
 // Code one lane's step (LE elements in v); when STORE, write its planes and
 // codes.  Returns escape flags: bit 4j for element j.
 template <int DT, bool STORE>
-__device__ __forceinline__ uint64_t code_step(const uint8_t *lut, uint4 v, int valid, const EPtr &q,
+__device__ __forceinline__ EMask<DT> code_step(uint32_t lut, uint4 v, int valid, const EPtr &q,
                                               int it) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     if constexpr (DT == SZ_BF16) {
@@ -218,8 +230,8 @@ __device__ __forceinline__ uint64_t code_step(const uint8_t *lut, uint4 v, int v
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const uint32_t ws = w[k] << 1;  // exponents in bytes 1 and 3
-            const uint32_t c0 = lut[__byte_perm(ws, 0, 0x4441)];
-            const uint32_t c1 = lut[ws >> 24];
+            const uint32_t c0 = lds_u8(lut + __byte_perm(ws, 0, 0x4441));
+            const uint32_t c1 = lds_u8(lut + (ws >> 24));
             cw += (c0 << (8 * k)) + (c1 << (8 * k + 4));
             // bytes 0 and 2: sign<<7 | mantissa of the two elements (bytes 1, 3 unused)
             x[k] = ((w[k] >> 8) & 0x00800080u) | (w[k] & 0xFF7FFF7Fu);
@@ -245,7 +257,7 @@ __device__ __forceinline__ uint64_t code_step(const uint8_t *lut, uint4 v, int v
         for (int k = 0; k < 4; ++k) {
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const uint32_t c = lut[(w[k] >> (8 * b + 2)) & 0x1Fu];
+                const uint32_t c = lds_u8(lut + ((w[k] >> (8 * b + 2)) & 0x1Fu));
                 cw[k >> 1] += c << (4 * (4 * (k & 1) + b));
             }
             if (STORE) {
@@ -293,14 +305,14 @@ __device__ __forceinline__ uint32_t exponent_at(uint4 v, uint32_t j) {
 
 // Rank one step's escapes within the block and hand each to put(rank, exponent).
 template <int DT, typename Put>
-__device__ __forceinline__ void rank_step(uint64_t m, uint4 v, uint32_t &running, Put put) {
-    const uint32_t c = __popcll(m);
+__device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &running, Put put) {
+    const uint32_t c = popc_mask(m);
     uint32_t tot;
     const uint32_t prefix = warp_exclusive_prefix(c, &tot);
     if (tot) {
         uint32_t r = running + prefix;
         while (m) {
-            const uint32_t j = uint32_t(__ffsll(m) - 1) >> 2;  // element, in element order
+            const uint32_t j = first_bit(m) >> 2;  // element, in element order
             m &= m - 1;
             put(r++, exponent_at<DT>(v, j));
         }
@@ -312,7 +324,7 @@ __device__ __forceinline__ void rank_step(uint64_t m, uint4 v, uint32_t &running
 // out; escapes (exponents in element order) go to put(rank, exponent).
 // Returns the block's escape count.
 template <int DT, bool STORE, typename Put>
-__device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t *in, uint64_t n,
+__device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, uint64_t n,
                                                uint64_t blk, const Layout &L, uint8_t *out, Put put) {
     using G = Geo<DT>;
     const int lane = threadIdx.x & 31;
@@ -320,6 +332,9 @@ __device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t
     const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
     const EPtr q = block_out<DT>(out, L, e_lane);
     uint32_t running = 0;
+    // pull the next block into L2 while this one is coded
+    if (STORE && lane == 0 && (blk + 2) * kBlock <= n)
+        prefetch_l2(in + (blk + 1) * kBlock * Dt<DT>::kElemBytes, kBlock * Dt<DT>::kElemBytes);
     if ((blk + 1) * kBlock <= n) {
         uint4 ring[G::kAhead + 1];
 #pragma unroll
@@ -330,7 +345,7 @@ __device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t
                 ring[(it + G::kAhead) % (G::kAhead + 1)] =
                     __ldcs(reinterpret_cast<const uint4 *>(src + (it + G::kAhead) * 512));
             const uint4 v = ring[it % (G::kAhead + 1)];
-            const uint64_t m = code_step<DT, STORE>(lut, v, G::LE, q, it);
+            const EMask<DT> m = code_step<DT, STORE>(lut, v, G::LE, q, it);
             rank_step<DT>(m, v, running, put);
         }
     } else {
@@ -338,7 +353,7 @@ __device__ __forceinline__ uint32_t code_block(const uint8_t *lut, const uint8_t
             const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
             const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
             const uint4 v = valid > 0 ? load_step<DT>(src + it * 512, valid) : make_uint4(0, 0, 0, 0);
-            const uint64_t m = code_step<DT, STORE>(lut, v, valid, q, it);
+            const EMask<DT> m = code_step<DT, STORE>(lut, v, valid, q, it);
             rank_step<DT>(m, v, running, put);
         }
     }
@@ -378,6 +393,9 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
     const uint8_t *in = p.in[t];
     uint8_t *out = p.out[t];
 
+    // pull the chunk's first block into L2 (a whole number of 16-byte units)
+    const uint32_t first_bytes = (uint32_t(min(uint64_t(kBlock), n - b0 * kBlock)) * Dt<DT>::kElemBytes) & ~15u;
+    if (lane == 0 && first_bytes) prefetch_l2(in + b0 * kBlock * Dt<DT>::kElemBytes, first_bytes);
     if (t != plan_tensor) {
         warp_load_plan<DT, MAXB>(p, t, W);
         plan_tensor = t;
@@ -391,13 +409,14 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
     const Layout L = stream_layout(DT, n, H.E);
 
     // ---- code the chunk's blocks; stage escapes in element order
+    const uint32_t lut = smem_u32(W.lut), stage = smem_u32(W.esc);
     uint32_t running = 0;
 #pragma unroll 1
     for (int k = 0; k < nbk; ++k) {
         if (lane == 0) W.blk_off[k] = running;
         const uint32_t base = running;
-        running += code_block<DT, true>(W.lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
-            if (base + r < kWarpStage) W.esc[base + r] = uint8_t(e);
+        running += code_block<DT, true>(lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+            if (base + r < kWarpStage) sts_u8(stage + base + r, e);
         });
     }
     __syncwarp();
@@ -423,7 +442,7 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
 #pragma unroll 1
         for (int k = 0; k < nbk; ++k) {
             const uint64_t d = dst + W.blk_off[k];
-            code_block<DT, false>(W.lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+            code_block<DT, false>(lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
                 if (d + r < L.total) out[d + r] = uint8_t(e);
             });
         }
@@ -448,7 +467,7 @@ __device__ void encode_empty(const EncodeParams<MAXB> &p, int t, WarpShared &W, 
 }
 
 template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT, 4) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
+__global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     __shared__ WarpShared s_warp[NW];
     __shared__ uint32_t s_epoch;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
