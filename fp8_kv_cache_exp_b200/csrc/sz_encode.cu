@@ -29,16 +29,21 @@ namespace {
 
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
-constexpr int kChunkBlocks = 4;                       // a warp's unit of work: 4 consecutive blocks
-constexpr uint32_t kWarpStage = 4096;                 // staged escape bytes per chunk
+constexpr int kChunkBlocks = 8;                       // a warp's unit of work: 8 consecutive blocks
+constexpr uint32_t kWarpStage = 2048;                 // staged escape bytes per chunk
+constexpr int kRing = 3;                              // quarter-block input stages per warp
+constexpr uint32_t kQuarterBytes = 2048;              // largest quarter block (BF16)
 constexpr int kLookbackPerLane = 4;                   // status words per lane per step
 constexpr uint64_t kLookbackLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
+constexpr uint64_t kWaitLimitNs = 1000000000ull;      // bulk-copy wait limit
 constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate published
 constexpr unsigned long long kFlagInc = 2ull << 32;   // inclusive prefix published
 
-// Each warp works alone: its own plan header, exponent -> code table and
-// escape stage.
-struct alignas(16) WarpShared {
+// Each warp works alone: its own input ring (bulk copies of quarter blocks),
+// plan header, exponent -> code table and escape stage.
+struct alignas(128) WarpShared {
+    uint8_t ring[kRing][kQuarterBytes];
+    uint64_t bar[kRing];
     uint32_t hdr[16];
     uint32_t blk_off[kChunkBlocks];  // escapes before each block, within the chunk
     uint8_t lut[256];
@@ -332,9 +337,6 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
     const EPtr q = block_out<DT>(out, L, e_lane);
     uint32_t running = 0;
-    // pull the next block into L2 while this one is coded
-    if (STORE && lane == 0 && (blk + 2) * kBlock <= n)
-        prefetch_l2(in + (blk + 1) * kBlock * Dt<DT>::kElemBytes, kBlock * Dt<DT>::kElemBytes);
     if ((blk + 1) * kBlock <= n) {
         uint4 ring[G::kAhead + 1];
 #pragma unroll
@@ -360,6 +362,45 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     return running;
 }
 
+// The warp's input ring: units are quarter blocks of the chunk being coded,
+// stage = unit % kRing; quarters of a partial (last) block are not copied and
+// are read from global memory instead.
+struct RingState {
+    uint32_t issued;  // bit s: stage s holds a copy not yet waited for
+    uint32_t parity;  // bit s: parity of stage s's next completion
+    uint32_t vi, vc;  // units issued / consumed
+};
+
+template <int DT>
+__device__ __forceinline__ void ring_issue(WarpShared &W, RingState &R, const uint8_t *in, uint64_t n,
+                                           uint64_t b0, uint32_t x) {
+    constexpr uint32_t kQB = kBlock / 4 * Dt<DT>::kElemBytes;  // bytes of a quarter block
+    const int st = int(R.vi % kRing);
+    const uint64_t blk = b0 + x / 4;
+    if ((blk + 1) * kBlock <= n) {
+        if ((threadIdx.x & 31) == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&W.bar[st], kQB);
+            bulk_g2s(W.ring[st], in + (blk * kBlock + (x % 4) * (kBlock / 4)) * Dt<DT>::kElemBytes, kQB,
+                     &W.bar[st]);
+        }
+        R.issued |= 1u << st;
+    }
+    ++R.vi;
+}
+
+// Wait for the unit about to be consumed; false if its copy never landed.
+__device__ __forceinline__ bool ring_take(WarpShared &W, RingState &R, int *stage) {
+    const int st = int(R.vc % kRing);
+    *stage = st;
+    ++R.vc;
+    if (!(R.issued & (1u << st))) return true;
+    const bool ok = mbar_wait(&W.bar[st], (R.parity >> st) & 1u, kWaitLimitNs);
+    R.parity ^= 1u << st;
+    R.issued &= ~(1u << st);
+    return ok;
+}
+
 // Load tensor t's plan into the warp's shared area and build its exponent ->
 // code table.
 template <int DT, int MAXB>
@@ -382,7 +423,7 @@ __device__ __forceinline__ void warp_load_plan(const EncodeParams<MAXB> &p, int 
 // One warp encodes chunk `chunk` (up to 4 blocks) of tensor t.
 template <int DT, int MAXB>
 __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t epoch,
-                             WarpShared &W, int &plan_tensor) {
+                             WarpShared &W, RingState &R, int &plan_tensor) {
     const int lane = threadIdx.x & 31;
     const int t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
     const uint32_t chunk = job - p.chunk_begin[t];
@@ -393,9 +434,6 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
     const uint8_t *in = p.in[t];
     uint8_t *out = p.out[t];
 
-    // pull the chunk's first block into L2 (a whole number of 16-byte units)
-    const uint32_t first_bytes = (uint32_t(min(uint64_t(kBlock), n - b0 * kBlock)) * Dt<DT>::kElemBytes) & ~15u;
-    if (lane == 0 && first_bytes) prefetch_l2(in + b0 * kBlock * Dt<DT>::kElemBytes, first_bytes);
     if (t != plan_tensor) {
         warp_load_plan<DT, MAXB>(p, t, W);
         plan_tensor = t;
@@ -408,17 +446,55 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
     }
     const Layout L = stream_layout(DT, n, H.E);
 
-    // ---- code the chunk's blocks; stage escapes in element order
+    // ---- code the chunk's blocks from the input ring; stage escapes in element order
+    using G = Geo<DT>;
+    constexpr int QIT = G::IT / 4;  // steps per quarter block
     const uint32_t lut = smem_u32(W.lut), stage = smem_u32(W.esc);
+    const uint32_t nunits = 4u * uint32_t(nbk);
+    uint32_t next_x = 0;
+    for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) ring_issue<DT>(W, R, in, n, b0, next_x);
     uint32_t running = 0;
+    bool lost = false;
 #pragma unroll 1
     for (int k = 0; k < nbk; ++k) {
+        const uint64_t blk = b0 + k;
         if (lane == 0) W.blk_off[k] = running;
+        const bool full = (blk + 1) * kBlock <= n;
+        const uint64_t e_lane = blk * kBlock + uint64_t(lane) * G::LE;
+        const EPtr q = block_out<DT>(out, L, e_lane);
         const uint32_t base = running;
-        running += code_block<DT, true>(lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+        auto put = [&](uint32_t r, uint32_t e) {
             if (base + r < kWarpStage) sts_u8(stage + base + r, e);
-        });
+        };
+        uint32_t blk_run = 0;
+#pragma unroll 1
+        for (int qq = 0; qq < 4; ++qq) {
+            if (next_x < nunits) ring_issue<DT>(W, R, in, n, b0, next_x++);
+            int st;
+            lost = !ring_take(W, R, &st) || lost;
+            if (full) {
+                const uint32_t src = smem_u32(W.ring[st]) + uint32_t(lane) * 16;
+#pragma unroll
+                for (int it = 0; it < QIT; ++it) {
+                    const uint4 v = lds_u128(src + it * 512);
+                    const EMask<DT> m = code_step<DT, true>(lut, v, G::LE, q, qq * QIT + it);
+                    rank_step<DT>(m, v, blk_run, put);
+                }
+            } else {
+                const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
+                for (int it = qq * QIT; it < (qq + 1) * QIT; ++it) {
+                    const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
+                    const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+                    const uint4 v = valid > 0 ? load_step<DT>(src + it * 512, valid) : make_uint4(0, 0, 0, 0);
+                    const EMask<DT> m = code_step<DT, true>(lut, v, valid, q, it);
+                    rank_step<DT>(m, v, blk_run, put);
+                }
+            }
+            __syncwarp();  // the stage just read may be refilled from here on
+        }
+        running += blk_run;
     }
+    if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
     __syncwarp();
 
     // ---- escape offset of the chunk within its tensor
@@ -467,14 +543,21 @@ __device__ void encode_empty(const EncodeParams<MAXB> &p, int t, WarpShared &W, 
 }
 
 template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
-    __shared__ WarpShared s_warp[NW];
+__global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
+    extern __shared__ __align__(128) uint8_t s_raw[];
+    WarpShared *s_warp = reinterpret_cast<WarpShared *>(s_raw);
     __shared__ uint32_t s_epoch;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
     __syncthreads();
     const uint32_t epoch = s_epoch;
     WarpShared &W = s_warp[warp];
+    if (lane == 0) {
+        for (int i = 0; i < kRing; ++i) mbar_init(&W.bar[i], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    RingState R = {0u, 0u, 0u, 0u};
     int plan_tensor = -1;
     // every warp claims chunks in launch order until none is left
     while (true) {
@@ -483,7 +566,7 @@ __global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ Enco
         job = __shfl_sync(0xffffffffu, job, 0);
         if (job >= p.total_jobs) break;
         if (job < p.total_chunks)
-            encode_chunk<DT, MAXB>(p, job, epoch, W, plan_tensor);
+            encode_chunk<DT, MAXB>(p, job, epoch, W, R, plan_tensor);
         else
             encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], W, plan_tensor);
     }
@@ -502,8 +585,11 @@ __global__ void __launch_bounds__(NT) encode_kernel(const __grid_constant__ Enco
 template <int DT, int MAXB>
 sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     auto kern = encode_kernel<DT, MAXB>;
+    const size_t smem = sizeof(WarpShared) * NW;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return SZ_ERR_CUDA;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, 0) != cudaSuccess || per_sm < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess || per_sm < 1)
         return SZ_ERR_CUDA;
     const uint64_t resident = uint64_t(a.num_sms) * per_sm;
     EncodeParams<MAXB> p;
@@ -512,7 +598,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     p.plans = a.plans;
     p.T = a.T;
     p.n_empty = 0;
-    p.chunk_log2 = 2;  // kChunkBlocks
+    p.chunk_log2 = 3;  // kChunkBlocks
     p.chunk_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
         p.in[t] = static_cast<const uint8_t *>(a.in[t]);
@@ -528,7 +614,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     if (p.total_jobs == 0) return SZ_OK;
     const uint64_t need = cdiv(p.total_jobs, NW);
     const uint64_t grid = need < resident ? need : resident;
-    kern<<<unsigned(grid), NT, 0, stream>>>(p);
+    kern<<<unsigned(grid), NT, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
 
