@@ -86,6 +86,36 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources and the C-ABI header (which kernels a profile describes)."""
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", "*")))
+    files.append(os.path.join(ROOT, "include", "splitzip.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by ncu for this kernel source, or None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = kernel_source_hash()
+    for line in lines:
+        parts = line.split()
+        if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                and parts[3] == src:
+            return int(parts[2])
+    return None
+
+
 def gpu_uuid(device) -> str:
     """nvidia-smi id of a torch device (its UUID, whatever CUDA_VISIBLE_DEVICES says)."""
     u = str(torch.cuda.get_device_properties(device).uuid)
@@ -258,8 +288,10 @@ def run_ours(args, rank, world, device):
         k["gbs"] = k["bytes"] / (k["ms"] * 1e-3) / 1e9
         k["frac"] = k["gbs"] / peak
     dom = max(kern, key=lambda k: kern[k]["ms"])
+    traffic = profiled_traffic(dom + "_kernel", wl.name) if world == 1 else None
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(kern[dom]["gbs"], 1), "peak": peak,
-            "unit": "GB/s", "frac": round(kern[dom]["frac"], 4), "traffic": None,
+            "unit": "GB/s", "frac": round(kern[dom]["frac"], 4),
+            "traffic": traffic, "algorithmic_bytes": kern[dom]["bytes"],
             "peak_source": peak_kind}
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT,
