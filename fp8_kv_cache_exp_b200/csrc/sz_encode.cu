@@ -30,7 +30,7 @@ namespace {
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
 constexpr int kChunkBlocks = 8;                       // a warp's unit of work: 8 consecutive blocks
-constexpr uint32_t kWarpStage = 2048;                 // staged escape bytes per chunk
+constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per chunk (two chunks)
 constexpr int kRing = 3;                              // quarter-block input stages per warp
 constexpr uint32_t kQuarterBytes = 2048;              // largest quarter block (BF16)
 constexpr int kLookbackPerLane = 4;                   // status words per lane per step
@@ -40,14 +40,15 @@ constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate publish
 constexpr unsigned long long kFlagInc = 2ull << 32;   // inclusive prefix published
 
 // Each warp works alone: its own input ring (bulk copies of quarter blocks),
-// plan header, exponent -> code table and escape stage.
+// plan header, exponent -> code table, and two escape stages (the chunk being
+// coded and one whose offset is still being looked up).
 struct alignas(128) WarpShared {
     uint8_t ring[kRing][kQuarterBytes];
     uint64_t bar[kRing];
     uint32_t hdr[16];
-    uint32_t blk_off[kChunkBlocks];  // escapes before each block, within the chunk
+    uint32_t blk_off[2][kChunkBlocks];  // escapes before each block, within the chunk
     uint8_t lut[256];
-    uint8_t esc[kWarpStage];
+    uint8_t esc[2][kWarpStage];
 };
 
 template <int DT>
@@ -57,31 +58,42 @@ struct Geo {
     static constexpr int kAhead = 3;                        // steps of loads in flight
 };
 
-// Decoupled look-back, run by one warp.  Returns the escapes in the tensor's
-// chunks before `chunk`; publishes this chunk's aggregate at once and its
-// inclusive prefix when known.  Status word: epoch (30 bits) << 34 |
-// flag << 32 | value; words of earlier launches carry an older epoch and read
-// as "not published".  Lane l reads positions 4l..4l+3 behind the cursor
-// (position 0 = nearest predecessor).
-__device__ uint32_t lookback(unsigned long long *st, uint32_t chunk, uint32_t agg, uint32_t epoch,
-                             bool *timed_out) {
+// Decoupled look-back of one chunk, run by one warp and resumable: the warp
+// publishes the chunk's aggregate, then sums its predecessors' published
+// values back to the nearest inclusive prefix.  Status word: epoch (30 bits)
+// << 34 | flag << 32 | value; words of earlier launches carry an older epoch
+// and read as "not published".  Lane l reads positions 4l..4l+3 behind the
+// cursor (position 0 = nearest predecessor).  Every predecessor publishes its
+// aggregate as soon as it has coded its chunk, without waiting on anything, so
+// a look-back always ends; the total wait is still bounded (SZ_ERR_TIMEOUT).
+struct Lookback {
+    int32_t j;      // nearest predecessor not yet summed
+    uint32_t excl;  // escapes summed so far
+    uint32_t t0;    // low bits of the time a predecessor was first found unpublished
+    uint32_t flags; // kLbDone | kLbTimedOut | kLbWaiting
+};
+constexpr uint32_t kLbDone = 1, kLbTimedOut = 2, kLbWaiting = 4;
+
+__device__ __forceinline__ void lookback_start(Lookback &lb, unsigned long long *st, uint32_t chunk,
+                                               uint32_t agg, unsigned long long tag) {
+    lb.j = int32_t(chunk) - 1;
+    lb.excl = 0;
+    lb.t0 = 0;
+    lb.flags = chunk == 0 ? kLbDone : 0u;
+    if ((threadIdx.x & 31) == 0) st_relaxed_u64(st + chunk, tag | (chunk == 0 ? kFlagInc : kFlagAgg) | agg);
+}
+
+// Sum published predecessors of chunk (status words st, own count agg); with
+// `block`, wait until done.  Returns true once the chunk's offset is known.
+__device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t chunk, uint32_t agg,
+                                 unsigned long long tag, bool block) {
     const int lane = threadIdx.x & 31;
-    const unsigned long long tag = (unsigned long long)(epoch & 0x3FFFFFFFu) << 34;
-    *timed_out = false;
-    if (chunk == 0) {
-        if (lane == 0) st_relaxed_u64(st, tag | kFlagInc | agg);
-        return 0;
-    }
-    if (lane == 0) st_relaxed_u64(st + chunk, tag | kFlagAgg | agg);
-    uint32_t excl = 0;
-    int64_t j = int64_t(chunk) - 1;
-    uint64_t t0 = 0;
     uint32_t backoff = 32;
-    while (true) {
+    while (!(lb.flags & kLbDone)) {
         uint32_t f[kLookbackPerLane], v[kLookbackPerLane];
 #pragma unroll
         for (int q = 0; q < kLookbackPerLane; ++q) {
-            const int64_t idx = j - kLookbackPerLane * lane - q;
+            const int32_t idx = lb.j - kLookbackPerLane * lane - q;
             f[q] = 2;  // before chunk 0: a virtual inclusive prefix of 0
             v[q] = 0;
             if (idx >= 0) {
@@ -107,23 +119,28 @@ __device__ uint32_t lookback(unsigned long long *st, uint32_t chunk, uint32_t ag
             }
         }
         if (__all_sync(0xffffffffu, ready)) {
-            excl += __reduce_add_sync(0xffffffffu, sum);
-            if (L < 32) break;
-            j -= 32 * kLookbackPerLane;
+            lb.excl += __reduce_add_sync(0xffffffffu, sum);
+            if (L < 32) {
+                lb.flags |= kLbDone;
+                break;
+            }
+            lb.j -= 32 * kLookbackPerLane;
             continue;
         }
-        const uint64_t now = __shfl_sync(0xffffffffu, global_ns(), 0);
-        if (t0 == 0) {
-            t0 = now;
-        } else if (now - t0 > kLookbackLimitNs) {
-            *timed_out = true;
+        const uint32_t now = __shfl_sync(0xffffffffu, uint32_t(global_ns()), 0);
+        if (!(lb.flags & kLbWaiting)) {
+            lb.flags |= kLbWaiting;
+            lb.t0 = now;
+        } else if (now - lb.t0 > uint32_t(kLookbackLimitNs)) {  // unsigned: correct across wrap
+            lb.flags |= kLbDone | kLbTimedOut;
             break;
         }
+        if (!block) return false;
         __nanosleep(backoff);
         if (backoff < 256) backoff <<= 1;
     }
-    if (lane == 0) st_relaxed_u64(st + chunk, tag | kFlagInc | (excl + agg));
-    return excl;
+    if (chunk != 0 && lane == 0) st_relaxed_u64(st + chunk, tag | kFlagInc | (lb.excl + agg));
+    return true;
 }
 
 template <int DT>
@@ -420,45 +437,61 @@ __device__ __forceinline__ void warp_load_plan(const EncodeParams<MAXB> &p, int 
     __syncwarp();
 }
 
-// One warp encodes chunk `chunk` (up to 4 blocks) of tensor t.
-template <int DT, int MAXB>
-__device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t epoch,
-                             WarpShared &W, RingState &R, int &plan_tensor) {
-    const int lane = threadIdx.x & 31;
-    const int t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
-    const uint32_t chunk = job - p.chunk_begin[t];
-    const uint64_t n = p.n[t];
-    const uint64_t nb = cdiv(n, kBlock);
-    const uint64_t b0 = uint64_t(chunk) * kChunkBlocks;
-    const int nbk = int(min(uint64_t(kChunkBlocks), nb - b0));
-    const uint8_t *in = p.in[t];
-    uint8_t *out = p.out[t];
+// Geometry of a chunk (job) of the launch.
+struct ChunkGeo {
+    int t;
+    uint32_t chunk;
+    uint64_t n, nb, b0;
+    int nbk;
+};
 
-    if (t != plan_tensor) {
-        warp_load_plan<DT, MAXB>(p, t, W);
-        plan_tensor = t;
+template <int MAXB>
+__device__ __forceinline__ ChunkGeo chunk_geo(const EncodeParams<MAXB> &p, uint32_t job) {
+    ChunkGeo g;
+    g.t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
+    g.chunk = job - p.chunk_begin[g.t];
+    g.n = p.n[g.t];
+    g.nb = cdiv(g.n, kBlock);
+    g.b0 = uint64_t(g.chunk) * kChunkBlocks;
+    g.nbk = int(min(uint64_t(kChunkBlocks), g.nb - g.b0));
+    return g;
+}
+
+// One warp codes a chunk: planes and codes go out, escapes are staged in
+// esc[slot] (element order) with per-block offsets in blk_off[slot].  Between
+// blocks it calls between().  Returns the chunk's escape count, or
+// 0xFFFFFFFF if the plan does not fit the data (reported; nothing to finish).
+template <int DT, int MAXB, typename Between>
+__device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
+                               WarpShared &W, RingState &R, int &plan_tensor, bool *lost, Between between) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t *in = p.in[g.t];
+    uint8_t *out = p.out[g.t];
+    const uint64_t n = g.n, b0 = g.b0;
+    const int nbk = g.nbk;
+    if (g.t != plan_tensor) {
+        warp_load_plan<DT, MAXB>(p, g.t, W);
+        plan_tensor = g.t;
     }
     const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     uint32_t why = 0;
-    if (!header_ok<DT>(H, n, p.cap[t], &why)) {
-        if (lane == 0 && chunk == 0) set_error(p.ctl, why, uint32_t(t));
-        return;  // every chunk of this tensor takes this branch: no look-back waits on it
+    if (!header_ok<DT>(H, n, p.cap[g.t], &why)) {
+        if (lane == 0 && g.chunk == 0) set_error(p.ctl, why, uint32_t(g.t));
+        return 0xFFFFFFFFu;  // every chunk of this tensor takes this branch: no look-back waits on it
     }
     const Layout L = stream_layout(DT, n, H.E);
 
-    // ---- code the chunk's blocks from the input ring; stage escapes in element order
     using G = Geo<DT>;
     constexpr int QIT = G::IT / 4;  // steps per quarter block
-    const uint32_t lut = smem_u32(W.lut), stage = smem_u32(W.esc);
+    const uint32_t lut = smem_u32(W.lut), stage = smem_u32(W.esc[slot]);
     const uint32_t nunits = 4u * uint32_t(nbk);
     uint32_t next_x = 0;
     for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) ring_issue<DT>(W, R, in, n, b0, next_x);
     uint32_t running = 0;
-    bool lost = false;
 #pragma unroll 1
     for (int k = 0; k < nbk; ++k) {
         const uint64_t blk = b0 + k;
-        if (lane == 0) W.blk_off[k] = running;
+        if (lane == 0) W.blk_off[slot][k] = running;
         const bool full = (blk + 1) * kBlock <= n;
         const uint64_t e_lane = blk * kBlock + uint64_t(lane) * G::LE;
         const EPtr q = block_out<DT>(out, L, e_lane);
@@ -471,7 +504,7 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
         for (int qq = 0; qq < 4; ++qq) {
             if (next_x < nunits) ring_issue<DT>(W, R, in, n, b0, next_x++);
             int st;
-            lost = !ring_take(W, R, &st) || lost;
+            *lost = !ring_take(W, R, &st) || *lost;
             if (full) {
                 const uint32_t src = smem_u32(W.ring[st]) + uint32_t(lane) * 16;
 #pragma unroll
@@ -493,38 +526,47 @@ __device__ void encode_chunk(const EncodeParams<MAXB> &p, uint32_t job, uint32_t
             __syncwarp();  // the stage just read may be refilled from here on
         }
         running += blk_run;
+        between();
     }
-    if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
     __syncwarp();
+    return running;
+}
 
-    // ---- escape offset of the chunk within its tensor
-    bool timed_out;
-    const uint32_t excl = lookback(p.status + p.chunk_begin[t], chunk, running, epoch, &timed_out);
+// Once the chunk's offset excl is known: its offsets-table entries, its
+// escapes (from the stage, or re-coded from the input when they overflowed
+// it -- the warp's code table is then still the chunk's), and the stream
+// frame if it is the tensor's last chunk.
+template <int DT, int MAXB>
+__device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
+                             uint32_t total, const Lookback &lb, WarpShared &W) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t *hdr = p.plans + 64 * size_t(g.t);
+    const Header H = load_header(hdr);
+    const Layout L = stream_layout(DT, g.n, H.E);
+    uint8_t *out = p.out[g.t];
+    const uint32_t excl = lb.excl;
     if (lane == 0) {
-        if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
-        if (uint64_t(excl) + running > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-        if (b0 + nbk == nb && uint64_t(excl) + running != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+        if (lb.flags & kLbTimedOut) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
+        if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+        if (g.b0 + g.nbk == g.nb && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
     }
-
-    // ---- offsets-table entries and escapes
-    if (lane < nbk) *reinterpret_cast<uint32_t *>(out + 64 + 4 * (b0 + lane)) = excl + W.blk_off[lane];
+    if (lane < g.nbk) *reinterpret_cast<uint32_t *>(out + 64 + 4 * (g.b0 + lane)) = excl + W.blk_off[slot][lane];
     const uint64_t dst = L.esc + excl;
-    if (running <= kWarpStage) {
-        __syncwarp();
-        for (uint32_t x = lane; x < running; x += 32)
-            if (dst + x < L.total) out[dst + x] = W.esc[x];
+    if (total <= kWarpStage) {
+        for (uint32_t x = lane; x < total; x += 32)
+            if (dst + x < L.total) out[dst + x] = W.esc[slot][x];
     } else {
-        // more escapes than the stage holds: re-read the chunk, write them directly
+        const uint32_t lut = smem_u32(W.lut);
 #pragma unroll 1
-        for (int k = 0; k < nbk; ++k) {
-            const uint64_t d = dst + W.blk_off[k];
-            code_block<DT, false>(lut, in, n, b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+        for (int k = 0; k < g.nbk; ++k) {
+            const uint64_t d = dst + W.blk_off[slot][k];
+            code_block<DT, false>(lut, p.in[g.t], g.n, g.b0 + k, L, out, [&](uint32_t r, uint32_t e) {
                 if (d + r < L.total) out[d + r] = uint8_t(e);
             });
         }
     }
-    if (b0 + nbk == nb) write_stream_frame(out, L, W.hdr, H.E);
-    __syncwarp();  // the stage may be refilled by the next chunk
+    if (g.b0 + g.nbk == g.nb) write_stream_frame(out, L, reinterpret_cast<const uint32_t *>(hdr), H.E);
+    __syncwarp();
 }
 
 // Stream of an empty tensor: header, offsets[0] = 0, zero padding (one warp).
@@ -542,6 +584,19 @@ __device__ void encode_empty(const EncodeParams<MAXB> &p, int t, WarpShared &W, 
     write_stream_frame(p.out[t], stream_layout(DT, 0, 0), W.hdr, 0);
 }
 
+// A chunk whose offset is still being looked up.
+struct Pending {
+    bool valid;
+    uint32_t job, total;
+    int slot;
+    Lookback lb;
+};
+
+template <int MAXB>
+__device__ __forceinline__ unsigned long long *chunk_status(const EncodeParams<MAXB> &p, int t) {
+    return p.status + p.chunk_begin[t];
+}
+
 template <int DT, int MAXB>
 __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     extern __shared__ __align__(128) uint8_t s_raw[];
@@ -551,6 +606,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
     if (tid == 0) s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
     __syncthreads();
     const uint32_t epoch = s_epoch;
+    const unsigned long long tag = (unsigned long long)(epoch & 0x3FFFFFFFu) << 34;
     WarpShared &W = s_warp[warp];
     if (lane == 0) {
         for (int i = 0; i < kRing; ++i) mbar_init(&W.bar[i], 1);
@@ -559,17 +615,50 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
     __syncwarp();
     RingState R = {0u, 0u, 0u, 0u};
     int plan_tensor = -1;
+    Pending pend;
+    pend.valid = false;
+    // finish the pending chunk once its look-back is done (blocking or not)
+    auto settle = [&](bool block) {
+        if (!pend.valid) return;
+        const ChunkGeo pg = chunk_geo<MAXB>(p, pend.job);
+        if (lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, block)) {
+            finish_chunk<DT, MAXB>(p, pend.job, pg, pend.slot, pend.total, pend.lb, W);
+            pend.valid = false;
+        }
+    };
     // every warp claims chunks in launch order until none is left
     while (true) {
         uint32_t job = 0;
         if (lane == 0) job = atomicAdd(&p.ctl[kCtlTileCtr], 1u);
         job = __shfl_sync(0xffffffffu, job, 0);
         if (job >= p.total_jobs) break;
-        if (job < p.total_chunks)
-            encode_chunk<DT, MAXB>(p, job, epoch, W, R, plan_tensor);
-        else
+        if (job >= p.total_chunks) {
             encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], W, plan_tensor);
+            continue;
+        }
+        const ChunkGeo g = chunk_geo<MAXB>(p, job);
+        const int slot = pend.valid ? (pend.slot ^ 1) : 0;
+        bool lost = false;
+        const uint32_t total = code_chunk<DT, MAXB>(p, job, g, slot, W, R, plan_tensor, &lost,
+                                                    [&]() { settle(false); });
+        if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
+        if (total == 0xFFFFFFFFu) continue;  // plan rejected for this tensor
+        unsigned long long *st = chunk_status(p, g.t);
+        Lookback lb;
+        lookback_start(lb, st, g.chunk, total, tag);
+        settle(true);  // at most one chunk waits for its offset
+        if (total > kWarpStage || lookback_advance(lb, st, g.chunk, total, tag, false)) {
+            lookback_advance(lb, st, g.chunk, total, tag, true);
+            finish_chunk<DT, MAXB>(p, job, g, slot, total, lb, W);
+        } else {
+            pend.valid = true;
+            pend.job = job;
+            pend.total = total;
+            pend.slot = slot;
+            pend.lb = lb;
+        }
     }
+    settle(true);
     // The last CTA to retire leaves the counters ready for the next launch.
     __syncthreads();
     if (tid == 0) {
