@@ -28,13 +28,18 @@ constexpr int kLargeBatch = SZ_MAX_BATCH;      // ... or for up to SZ_MAX_BATCH 
 
 // Control words at the start of every workspace (u32 each).
 enum : int {
-    kCtlErr = 0,       // first device error (sz_status), 0 if none
-    kCtlErrDetail = 1, // error detail (e.g. the tile that failed)
-    kCtlEpoch = 2,     // encode launch counter, tags look-back status words
-    kCtlTileCtr = 3,   // encode job counter (tile ids in launch order)
-    kCtlDone = 4,      // encode CTAs finished
-    kCtlWords = 64     // 256 bytes reserved
+    kCtlErr = 0,         // first device error (sz_status), 0 if none
+    kCtlErrDetail = 1,   // error detail (e.g. the tile that failed)
+    kCtlEpoch = 2,       // encode launch counter, tags look-back status words
+    kCtlTileCtr = 3,     // encode job counter (tile ids in launch order)
+    kCtlDone = 4,        // encode CTAs finished
+    kCtlDecodeDone = 5,  // decode CTAs finished
+    kCtlWords = 64       // 256 bytes reserved
 };
+// Decode's per-tensor block counters live in word 0 of each tensor's
+// histogram slot (plan leaves the histograms zero; decode zeroes its counters
+// before it returns), one 1 KB slot apart.
+constexpr uint32_t kClaimStride = 256;
 
 __host__ __device__ constexpr uint64_t align256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
 __host__ __device__ constexpr uint64_t cdiv(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
@@ -146,6 +151,7 @@ struct EncodeParams {
 template <int MAXB>
 struct DecodeParams {
     uint32_t *ctl;
+    uint32_t *claim;     // per-tensor block counters, word t * kClaimStride (zero between calls)
     uint32_t total_blocks;
     int T;
     const uint8_t *comp[MAXB];

@@ -5,9 +5,12 @@
 // time ...": decompression runs on the decode GPU.  The stored per-block
 // escape offsets make decode a pure gather with no dependency between blocks,
 // so one warp decodes one 4096-element block on its own, with no CTA barrier:
-//   - every warp owns a contiguous range of the launch's blocks, and checks a
-//     tensor's header (and builds its code-pair table) when it reaches it; a
-//     stream that fails a check sets SZ_ERR_CORRUPT_STREAM and is not written;
+//   - warps claim blocks one at a time from per-tensor counters (claiming the
+//     next block while decoding the current one), so they all finish within
+//     about one block of each other; a warp stays in one tensor while it has
+//     blocks and checks a tensor's header (and builds its code-pair table)
+//     when it moves to it; a stream that fails a check sets
+//     SZ_ERR_CORRUPT_STREAM and is not written;
 //   - the block's code and plane bytes (6 KB BF16, 3.5 KB E5M2) arrive by bulk
 //     copy into one of the warp's two shared-memory stages while the warp
 //     decodes the previous block (waits are bounded); the next block's
@@ -321,42 +324,94 @@ __device__ __forceinline__ uint32_t load_escape_reg(const uint8_t *comp, const W
     return (lane < cnt && b.hi <= ws.E) ? uint32_t(comp[ws.esc + b.lo + lane]) : 0u;
 }
 
-// The warp's quarter-block units in order; the producer side of its ring.
+template <int MAXB>
+__device__ __forceinline__ uint32_t nblocks(const DecodeParams<MAXB> &p, int t) {
+    return p.block_begin[t + 1] - p.block_begin[t];
+}
+
+// Warp-wide block claim.  `first` (valid in lane 0) is the result of an
+// atomicAdd that lane 0 already made on tensor t's counter; if that block
+// exists it is the claim.  Otherwise the other tensors are scanned, 32 per
+// step starting after t, and each one whose counter is still below its block
+// count is tried with an atomicAdd.  Returns the block and sets t to its
+// tensor; t = -1 once every tensor's blocks are taken (counters only grow, so
+// a tensor seen exhausted stays exhausted).
+template <int MAXB>
+__device__ __forceinline__ uint32_t claim_resolve(const DecodeParams<MAXB> &p, int &t, uint32_t first) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t r = __shfl_sync(0xffffffffu, first, 0);
+    if (r < nblocks(p, t)) return r;
+    for (int base = 1; base <= p.T; base += 32) {
+        const int k = base + lane;  // tensors t+1 .. t+T (mod T), t itself last
+        int u = 0;
+        bool open = false;
+        if (k <= p.T) {
+            u = t + k >= p.T ? t + k - p.T : t + k;
+            open = ld_relaxed_u32(p.claim + u * kClaimStride) < nblocks(p, u);
+        }
+        uint32_t m = __ballot_sync(0xffffffffu, open);
+        while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            const int uu = __shfl_sync(0xffffffffu, u, src);
+            uint32_t rr = 0;
+            if (lane == 0) rr = atomicAdd(p.claim + uu * kClaimStride, 1u);
+            rr = __shfl_sync(0xffffffffu, rr, 0);
+            if (rr < nblocks(p, uu)) {
+                t = uu;
+                return rr;
+            }
+        }
+    }
+    t = -1;
+    return 0;
+}
+
+// The warp's quarter-block units in claim order; the producer side of its
+// ring.  It runs three units ahead of the consumer, so it reaches the next
+// block's first quarter while the consumer is on the current block's second:
+// the next block is handed over (set_next) just before that.
 template <int DT, int MAXB>
 struct QuarterFeed {
-    uint32_t g, g_end;  // block (launch-global) of the next unit to issue, end of range
-    int q, t;           // its quarter and tensor
+    static constexpr int kAwait = -2;
+    int t;          // tensor of the next unit to issue; -1: no more units, kAwait: next block not yet known
+    uint32_t blk;   // its block within the tensor
+    int q;          // its quarter
+    bool full;      // the block has all 4096 elements (partial blocks are read directly)
+    int sg_t;       // tensor whose geometry sg holds
     StreamGeo sg;
-    uint32_t v;         // units issued so far
+    uint32_t v;     // units issued so far
 
-    __device__ __forceinline__ void start(const DecodeParams<MAXB> &p, uint32_t b_lo, uint32_t b_hi, int t0) {
-        g = b_lo;
-        g_end = b_hi;
-        q = 0;
-        t = t0;
-        sg = stream_geo<DT, MAXB>(p, t);
+    __device__ __forceinline__ void start(const DecodeParams<MAXB> &p, int t0, uint32_t blk0) {
+        sg_t = -1;
         v = 0;
+        set_next(p, t0, blk0);
+    }
+    __device__ __forceinline__ void set_next(const DecodeParams<MAXB> &p, int tn, uint32_t bn) {
+        t = tn;
+        blk = bn;
+        q = 0;
+        full = false;
+        if (tn >= 0) {
+            if (tn != sg_t) {
+                sg = stream_geo<DT, MAXB>(p, tn);
+                sg_t = tn;
+            }
+            full = (uint64_t(bn) + 1) * kBlock <= p.n[tn];
+        }
     }
     // Issue the next unit into stage v % kStages (if it is part of a full
     // block); returns the bit to set in the issued mask.
-    __device__ __forceinline__ uint32_t issue_next(const DecodeParams<MAXB> &p, WarpSmem &W) {
-        if (g >= g_end) return 0;
-        if (p.block_begin[t + 1] <= g) {
-            while (p.block_begin[t + 1] <= g) ++t;
-            sg = stream_geo<DT, MAXB>(p, t);
-        }
-        const uint64_t blk = g - p.block_begin[t];
+    __device__ __forceinline__ uint32_t issue_next(WarpSmem &W) {
+        if (t < 0) return 0;
         const int st = int(v % kStages);
         uint32_t bit = 0;
-        if ((blk + 1) * kBlock <= p.n[t]) {
+        if (full) {
             if ((threadIdx.x & 31) == 0) issue_quarter<DT>(W.stage[st], &W.bar[st], sg, blk, q);
             bit = 1u << st;
         }
         ++v;
-        if (++q == 4) {
-            q = 0;
-            ++g;
-        }
+        if (++q == 4) t = kAwait;
         return bit;
     }
 };
@@ -374,95 +429,116 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
     }
     __syncwarp();
 
-    // every warp owns a contiguous range of the launch's blocks
+    // Blocks are claimed one at a time from per-tensor counters, one block
+    // ahead of the one being decoded.  Each warp starts in the tensor that
+    // holds its proportional share of the launch's blocks, stays there while
+    // it has blocks, then moves to any tensor that still has some.
     const uint64_t nwarps = uint64_t(gridDim.x) * NW;
     const uint64_t gw = uint64_t(blockIdx.x) * NW + warp;
-    const uint32_t b_lo = uint32_t(uint64_t(p.total_blocks) * gw / nwarps);
-    const uint32_t b_hi = uint32_t(uint64_t(p.total_blocks) * (gw + 1) / nwarps);
-    if (b_lo >= b_hi) return;
+    int t = find_tensor<uint32_t, MAXB>(p.block_begin, p.T, uint32_t(uint64_t(p.total_blocks) * gw / nwarps));
+    uint32_t first = 0;
+    if (lane == 0) first = atomicAdd(p.claim + t * kClaimStride, 1u);
+    uint32_t blk = claim_resolve<MAXB>(p, t, first);
 
-    int t = find_tensor<uint32_t, MAXB>(p.block_begin, p.T, b_lo);
-    QuarterFeed<DT, MAXB> feed;
-    feed.start(p, b_lo, b_hi, t);
     uint32_t issued = 0;  // bit s: stage s holds an issued unit not yet waited for
     uint32_t parity = 0;  // bit s: parity of stage s's next completion
-    for (int k = 0; k < kStages - 1; ++k) issued |= feed.issue_next(p, W);
+    if (t >= 0) {
+        QuarterFeed<DT, MAXB> feed;
+        feed.start(p, t, blk);
+        for (int k = 0; k < kStages - 1; ++k) issued |= feed.issue_next(W);
 
-    WarpStream ws;
-    warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
-    uint64_t blk = b_lo - p.block_begin[t];
-    BlockEsc be = load_offsets(p.comp[t], blk);
-    uint32_t esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
-    uint32_t v = 0;  // units consumed
+        WarpStream ws;
+        warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
+        BlockEsc be = load_offsets(p.comp[t], blk);
+        uint32_t esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
+        uint32_t v = 0;  // units consumed
 
-    for (uint32_t g = b_lo; g < b_hi; ++g) {
-        const uint8_t *comp = p.comp[t];
-        const bool next_same = g + 1 < b_hi && g + 1 < p.block_begin[t + 1];
-        BlockEsc be_n = {0, 0};
-        if (next_same && ws.ok) be_n = load_offsets(comp, blk + 1);
-        uint32_t esc_n = 0;
+        while (true) {
+            const uint8_t *comp = p.comp[t];
+            uint32_t pend = 0;  // claim of the next block, resolved at the second quarter
+            if (lane == 0) pend = atomicAdd(p.claim + t * kClaimStride, 1u);
+            int t_n = t;
+            uint32_t blk_n = 0;
+            BlockEsc be_n = {0, 0};
+            uint32_t esc_n = 0;
 
-        const bool ok = ws.ok && offsets_ok(be, ws, blk);
-        const uint32_t cnt = ok ? be.hi - be.lo : 0u;
-        const uint8_t *esc_g = comp + ws.esc + be.lo;
-        uint8_t *out = p.out[t] + (blk * kBlock + uint64_t(lane) * G::LE) * Dt<DT>::kElemBytes;
-        const bool full = (blk + 1) * kBlock <= ws.n;
-        uint32_t running = 0;
-        bool bad = false, timed_out = false;
-        for (int q = 0; q < 4; ++q, ++v) {
-            issued |= feed.issue_next(p, W);
-            const int st = int(v % kStages);
-            if (issued & (1u << st)) {
-                timed_out = timed_out || !mbar_wait(&W.bar[st], (parity >> st) & 1u, kWaitLimitNs);
-                parity ^= 1u << st;
-                issued &= ~(1u << st);
-            }
-            if (q == 1 && next_same && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
-            if (ok && !timed_out) {
-                if (full) {
-                    const uint32_t st_addr = smem_u32(W.stage[st]);
+            const bool ok = ws.ok && offsets_ok(be, ws, blk);
+            const uint32_t cnt = ok ? be.hi - be.lo : 0u;
+            const uint8_t *esc_g = comp + ws.esc + be.lo;
+            uint8_t *out = p.out[t] + (uint64_t(blk) * kBlock + uint64_t(lane) * G::LE) * Dt<DT>::kElemBytes;
+            const bool full = (uint64_t(blk) + 1) * kBlock <= ws.n;
+            uint32_t running = 0;
+            bool bad = false, timed_out = false;
+            for (int q = 0; q < 4; ++q, ++v) {
+                if (q == 1) {
+                    blk_n = claim_resolve<MAXB>(p, t_n, pend);
+                    feed.set_next(p, t_n, blk_n);
+                    if (t_n == t && ws.ok) be_n = load_offsets(comp, blk_n);
+                }
+                issued |= feed.issue_next(W);
+                const int st = int(v % kStages);
+                if (issued & (1u << st)) {
+                    timed_out = timed_out || !mbar_wait(&W.bar[st], (parity >> st) & 1u, kWaitLimitNs);
+                    parity ^= 1u << st;
+                    issued &= ~(1u << st);
+                }
+                if (q == 2 && t_n == t && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
+                if (ok && !timed_out) {
+                    if (full) {
+                        const uint32_t st_addr = smem_u32(W.stage[st]);
 #pragma unroll
-                    for (int it = 0; it < G::QIT; ++it) {
-                        const DFrag f = read_stage<DT>(st_addr, it);
-                        decode_step<DT, false>(f, tab_addr, out + (q * G::QIT + it) * 512, G::LE, running,
-                                               esc_reg, esc_g, cnt, bad);
-                    }
-                } else {
-                    for (int it = q * G::QIT; it < (q + 1) * G::QIT; ++it) {
-                        const int64_t e = int64_t(blk * kBlock) + int64_t(it) * 32 * G::LE + int64_t(lane) * G::LE;
-                        const int64_t left = int64_t(ws.n) - e;
-                        const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
-                        const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
-                        decode_step<DT, true>(f, tab_addr, out + it * 512, valid, running, esc_reg, esc_g, cnt, bad);
+                        for (int it = 0; it < G::QIT; ++it) {
+                            const DFrag f = read_stage<DT>(st_addr, it);
+                            decode_step<DT, false>(f, tab_addr, out + (q * G::QIT + it) * 512, G::LE, running,
+                                                   esc_reg, esc_g, cnt, bad);
+                        }
+                    } else {
+                        for (int it = q * G::QIT; it < (q + 1) * G::QIT; ++it) {
+                            const int64_t e = int64_t(blk) * kBlock + int64_t(it) * 32 * G::LE + int64_t(lane) * G::LE;
+                            const int64_t left = int64_t(ws.n) - e;
+                            const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+                            const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
+                            decode_step<DT, true>(f, tab_addr, out + it * 512, valid, running, esc_reg, esc_g, cnt,
+                                                  bad);
+                        }
                     }
                 }
+                __syncwarp();  // the stage just read may be refilled from here on
             }
-            __syncwarp();  // the stage just read may be refilled from here on
-        }
-        if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
-        if (lane == 0) {
-            if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, g);
-            else if (ws.ok && (!ok || bad)) set_error(p.ctl, SZ_ERR_CORRUPT_STREAM, g);
-        }
-        if (timed_out) return;  // a copy that never lands: stop this warp
+            if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
+            if (lane == 0) {
+                const uint32_t g = p.block_begin[t] + blk;
+                if (timed_out) set_error(p.ctl, SZ_ERR_TIMEOUT, g);
+                else if (ws.ok && (!ok || bad)) set_error(p.ctl, SZ_ERR_CORRUPT_STREAM, g);
+            }
+            if (timed_out || t_n < 0) break;  // a copy that never landed stops this warp
 
-        // ---- advance
-        if (g + 1 >= b_hi) break;
-        if (next_same) {
-            ++blk;
-            be = be_n;
-            esc_reg = esc_n;
-        } else {
-            while (p.block_begin[t + 1] <= g + 1) ++t;
-            warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
-            blk = 0;
-            be = load_offsets(p.comp[t], blk);
-            esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
+            // ---- advance to the claimed block
+            if (t_n == t) {
+                be = be_n;
+                esc_reg = esc_n;
+            } else {
+                t = t_n;
+                warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
+                be = load_offsets(p.comp[t], blk_n);
+                esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
+            }
+            blk = blk_n;
         }
     }
     // wait for copies still in flight before the warp's shared memory goes away
     for (int st = 0; st < kStages; ++st)
         if (issued & (1u << st)) mbar_wait(&W.bar[st], (parity >> st) & 1u, kWaitLimitNs);
+
+    // the last CTA out zeroes the claim counters for the next call
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&p.ctl[kCtlDecodeDone], 1u) == gridDim.x - 1) {
+            for (int u = 0; u < p.T; ++u) atomicExch(p.claim + u * kClaimStride, 0u);
+            atomicExch(&p.ctl[kCtlDecodeDone], 0u);
+        }
+    }
 }
 
 template <int DT, int MAXB>
@@ -476,6 +552,7 @@ sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
         return SZ_ERR_CUDA;
     DecodeParams<MAXB> p;
     p.ctl = a.ctl;
+    p.claim = a.ctl + kCtlWords;  // the histogram slots
     p.T = a.T;
     p.block_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {

@@ -120,3 +120,36 @@ def test_workspace_reuse_is_deterministic():
     y = x.view(-1)[: 4096 * 5]
     gpu_encode(0, y, ws)
     assert np.array_equal(gpu_encode(0, x, ws)[1], first)
+
+
+def test_batched_decode_claims_every_block_and_resets():
+    """Decode hands blocks out from per-tensor counters in the workspace: with
+    more tensors than one warp scans at a time (empty and one-element tensors
+    among them), every block is decoded exactly right, the counters are zero
+    again after each call, and plan can reuse the workspace straight away."""
+    m = sz()
+    rng = np.random.default_rng(21)
+    for dtype in (0, 1):
+        sizes = [int(s) for s in rng.choice([0, 1, 4095, 4096, 4097, 3 * 4096 + 5, 9 * 4096, 40000], 70)]
+        raws = [oracle_pins._kvlike(rng, n, dtype) for n in sizes]
+        xs = [from_raw(r, dtype) for r in raws]
+        ws = m.new_workspace(dtype, sizes)
+        plans = m.new_plans(len(xs))
+        m.sz_plan_batched(dtype, xs, ws, plans)
+        totals = m.sz_compressed_sizes(plans)
+        outs = [torch.zeros(m.sz_max_compressed_size(dtype, n), dtype=torch.uint8, device="cuda") for n in sizes]
+        m.sz_encode_batched(dtype, plans, xs, outs, ws)
+        assert m.sz_last_device_status(ws) == 0
+        for rep in range(3):
+            decs = [torch.full_like(x.view(torch.uint8), 0xA5) for x in xs]
+            m.sz_decode_batched(dtype, [o[:t] for o, t in zip(outs, totals)],
+                                [d.view(x.dtype) for d, x in zip(decs, xs)], ws)
+            assert m.sz_last_device_status(ws) == 0
+            words = ws.view(torch.int32)
+            assert words[5].item() == 0
+            assert not words[64: 64 + 256 * len(sizes)].any().item(), "claim counters left set"
+            for raw, dec in zip(raws, decs):
+                assert np.array_equal(dec.cpu().numpy(), raw)
+        plans2 = m.new_plans(len(xs))
+        m.sz_plan_batched(dtype, xs, ws, plans2)
+        assert torch.equal(plans2, plans)
