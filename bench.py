@@ -176,12 +176,14 @@ class ClockSampler:
 # ------------------------------------------------------------- our arm
 
 class Workload:
-    def __init__(self, name: str, rank: int, world: int, device):
+    def __init__(self, name: str, rank: int, world: int, device, layers=None):
         cfg_name, layers_per_step, desc = WORKLOADS[name]
         self.name, self.desc = name, desc
         self.cfg = kvgen.CONFIGS[cfg_name]
         self.dtype = 1 if self.cfg.fp8 else 0
         nl = self.cfg.layers if layers_per_step is None else layers_per_step
+        if layers is not None:  # a smaller batch of the same tensors (profiler captures)
+            nl = layers
         self.layers = rank_layers(nl, rank, world)
         self.xs = [kvgen.kv_tensor(self.cfg, l % self.cfg.layers if world == 1 else l, kv, device=device)
                    for l in self.layers for kv in (0, 1)]
@@ -192,7 +194,7 @@ class Workload:
 
 def run_ours(args, rank, world, device):
     import fp8_kv_cache_exp_b200 as sz
-    wl = Workload(args.workload, rank, world, device)
+    wl = Workload(args.workload, rank, world, device, args.layers)
     dt = wl.dtype
     T = len(wl.xs)
     stream = torch.cuda.current_stream()
@@ -439,6 +441,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3-8b")
     ap.add_argument("--mode", choices=["batch", "per_layer"], default="batch")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step (default: the workload's); smaller batches are for profiler captures")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     args = ap.parse_args()

@@ -299,6 +299,17 @@ __device__ inline int find_tensor(const U (&begin)[MAXB + 1], int T, U x) {
     return lo;
 }
 
+// prmt.b32 in its default mode (PTX ISA, "prmt"): byte i of the result is
+// byte (s_i & 7) of the pair {b, a} (a = bytes 0-3) when selector nibble s_i
+// (bits 4i..4i+3 of s) is below 8, and that byte's top bit copied into all
+// 8 bits when s_i >= 8.  Four table lookups of up to 8 bytes in one
+// instruction.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+    return d;
+}
+
 // Exclusive prefix of c over the lanes of a warp; *total receives the warp's
 // sum.  When no lane has c > 1 (escapes are rare) the prefix is a popcount of
 // the lanes below with c = 1; otherwise a shuffle scan.

@@ -69,6 +69,7 @@ struct WarpStream {
     uint32_t nb;                  // 4096-element blocks
     uint64_t n, E;
     uint64_t code, pa, pb, esc;   // section offsets in the stream
+    uint32_t xt[4];               // E5M2: byte c = exponent of code c, times 4 (byte 15: 0)
 };
 
 // Step `it` (within a quarter block) from the shared-memory stage at address st.
@@ -131,9 +132,10 @@ __device__ __forceinline__ DFrag read_partial(const uint8_t *comp, const WarpStr
     return f;
 }
 
-// Check tensor t's header with the warp; on success fill the code-pair table:
-// tab[b] = exponents of the two codes in byte b, pre-spread for reassembly
-// (BF16: e_even | e_odd << 16; E5M2: e_even | e_odd << 8); code 15 gives 0.
+// Check tensor t's header with the warp; on success fill the code tables.
+// BF16: the shared code-pair table, tab[b] = exponents of the two codes in
+// byte b pre-spread for reassembly (e_even | e_odd << 16); E5M2: the register
+// table ws.xt.  Code 15 gives 0 in both.
 template <int DT, int MAXB>
 __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, int t, uint32_t *tab, WarpStream &ws) {
     const int lane = threadIdx.x & 31;
@@ -162,12 +164,12 @@ __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, in
         const bool dtype_mismatch = w[0] == kMagic && ((w[1] >> 16) & 0xFFu) != uint32_t(DT);
         set_error(p.ctl, dtype_mismatch ? SZ_ERR_UNSUPPORTED_DTYPE : SZ_ERR_CORRUPT_STREAM, uint32_t(t));
     }
-    if (ok) {
+    if (ok && DT == SZ_BF16) {
         for (int b = lane; b < 256; b += 32) {
             const uint32_t c0 = b & 15, c1 = b >> 4;
             const uint32_t e0 = c0 < kCodes ? cb_byte(cbw, int(c0)) : 0u;
             const uint32_t e1 = c1 < kCodes ? cb_byte(cbw, int(c1)) : 0u;
-            tab[b] = (DT == SZ_BF16) ? (e0 | (e1 << 16)) : (e0 | (e1 << 8));
+            tab[b] = e0 | (e1 << 16);
         }
     }
     __syncwarp();
@@ -181,6 +183,10 @@ __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, in
     ws.pa = L.plane[0];
     ws.pb = L.plane[1];
     ws.esc = L.esc;
+    // E5M2 exponents are below 32, so every byte of the x4 table stays below
+    // 128: a selector nibble with its top bit set reads as zero (see prmt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ws.xt[i] = ok ? (cbw[i] << 2) : 0u;
 }
 
 // Section offsets of a tensor's stream; they depend on n only.
@@ -234,8 +240,8 @@ __device__ __forceinline__ void patch(uint32_t (&o)[4], uint32_t j, uint32_t e) 
 // esc_reg: lane i holds the block's escape i (i < 32); esc_g: the block's
 // escapes in global memory; cnt: escapes the offsets table gives the block.
 template <int DT, bool PARTIAL>
-__device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, uint8_t *dst,
-                                            int valid, uint32_t &running, uint32_t esc_reg,
+__device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const uint32_t (&xt)[4],
+                                            uint8_t *dst, int valid, uint32_t &running, uint32_t esc_reg,
                                             const uint8_t *esc_g, uint32_t cnt, bool &bad) {
     uint32_t o[4];
     // escape flags of this lane's elements: bit 4j for element j
@@ -250,24 +256,46 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, uint8_
         }
         m = escape_nibbles(cw);
     } else {
+        // four codes per word select their exponents from the register table:
+        // codes 0-7 from bytes 0-7, codes 8-15 from bytes 8-15 (selector with
+        // the top bit flipped, so each half reads zero for the other's codes)
+        const uint32_t x0 = f.c0 ^ 0x88888888u, x1 = f.c1 ^ 0x88888888u;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const uint32_t cw = (k < 2) ? f.c0 : f.c1;
-            const uint32_t lo = lds_u32(tab + (((cw >> (16 * (k & 1))) & 0xFFu) << 2));
-            const uint32_t hi = lds_u32(tab + (((cw >> (16 * (k & 1) + 8)) & 0xFFu) << 2));
-            const uint32_t e4 = lo | (hi << 16);
+            const uint32_t cw = (k < 2) ? f.c0 : f.c1, cx = (k < 2) ? x0 : x1;
+            const uint32_t sl = (k & 1) ? (cw >> 16) : cw, sh = (k & 1) ? (cx >> 16) : cx;
+            const uint32_t e4 = prmt(xt[0], xt[1], sl) | prmt(xt[2], xt[3], sh);
             const uint32_t s4 = (f.a >> (4 * k)) & 0xFu;
             const uint32_t sgn = (s4 * 0x10204080u) & 0x80808080u;
-            const uint32_t m8 = (f.b >> (8 * k)) & 0xFFu;
-            const uint32_t mnt = (m8 | (m8 << 6) | (m8 << 12) | (m8 << 18)) & 0x03030303u;
-            o[k] = (sgn | mnt) + (e4 << 2);
+            // 2-bit mantissas of the four elements (byte k of plane b) to bits 0-1 of each byte
+            const uint32_t m8 = prmt(f.b, 0u, 0x4440u + uint32_t(k));
+            const uint32_t t = (m8 | (m8 << 12)) & 0x000F000Fu;
+            const uint32_t mnt = (t | (t << 6)) & 0x03030303u;
+            o[k] = sgn | mnt | e4;
         }
         m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
     }
     const uint32_t c = (DT == SZ_BF16) ? uint32_t(__popc(uint32_t(m))) : uint32_t(__popcll(uint64_t(m)));
-    uint32_t tot;
-    const uint32_t prefix = warp_exclusive_prefix(c, &tot);
-    if (tot) {
+    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+    if (any == 0) {
+        // no escape in this step
+    } else if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+        // at most one escape per lane: its rank counts the lanes before it that have one
+        const uint32_t lane = threadIdx.x & 31;
+        const uint32_t r = running + __popc(any & ((1u << lane) - 1u));
+        const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
+        if (c) {
+            const uint32_t j = uint32_t((DT == SZ_BF16) ? __ffs(uint32_t(m)) - 1 : __ffsll(uint64_t(m)) - 1) >> 2;
+            uint32_t e = 0;
+            if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
+            else bad = true;
+            if (DT == SZ_FP8_E5M2 && e >= 32u) bad = true;
+            patch<DT>(o, j, e & (Dt<DT>::kBins - 1));
+        }
+        running += __popc(any);
+    } else {
+        uint32_t tot;
+        const uint32_t prefix = warp_exclusive_prefix(c, &tot);
         const uint32_t maxc = __reduce_max_sync(0xffffffffu, c);
         auto mm = m;
         for (uint32_t i = 0; i < maxc; ++i) {
@@ -489,7 +517,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
 #pragma unroll
                         for (int it = 0; it < G::QIT; ++it) {
                             const DFrag f = read_stage<DT>(st_addr, it);
-                            decode_step<DT, false>(f, tab_addr, out + (q * G::QIT + it) * 512, G::LE, running,
+                            decode_step<DT, false>(f, tab_addr, ws.xt, out + (q * G::QIT + it) * 512, G::LE, running,
                                                    esc_reg, esc_g, cnt, bad);
                         }
                     } else {
@@ -498,7 +526,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
                             const int64_t left = int64_t(ws.n) - e;
                             const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
                             const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
-                            decode_step<DT, true>(f, tab_addr, out + it * 512, valid, running, esc_reg, esc_g, cnt,
+                            decode_step<DT, true>(f, tab_addr, ws.xt, out + it * 512, valid, running, esc_reg, esc_g, cnt,
                                                   bad);
                         }
                     }

@@ -47,7 +47,7 @@ struct alignas(128) WarpShared {
     uint64_t bar[kRing];
     uint32_t hdr[16];
     uint32_t blk_off[2][kChunkBlocks];  // escapes before each block, within the chunk
-    uint8_t lut[256];
+    uint8_t lut_raw[512];  // holds the 256-byte-aligned code table (lut_addr)
     uint8_t esc[2][kWarpStage];
 };
 
@@ -236,6 +236,14 @@ __device__ __forceinline__ EPtr block_out(uint8_t *out, const Layout &L, uint64_
 template <int DT>
 using EMask = typename std::conditional<DT == SZ_BF16, uint32_t, uint64_t>::type;
 
+// Shared address of the warp's code table: 256 one-byte entries starting on a
+// 256-byte boundary, so that one prmt forms an entry's address from the table
+// address (bytes 1-3) and an index byte of the data (byte 0).  BF16 entries
+// are indexed by the exponent, E5M2 entries by the whole element byte.
+__device__ __forceinline__ uint32_t lut_addr(const WarpShared &W) {
+    return (smem_u32(W.lut_raw) + 255u) & ~255u;
+}
+
 __device__ __forceinline__ uint32_t popc_mask(uint32_t m) { return __popc(m); }
 __device__ __forceinline__ uint32_t popc_mask(uint64_t m) { return __popcll(m); }
 __device__ __forceinline__ uint32_t first_bit(uint32_t m) { return __ffs(m) - 1; }
@@ -252,8 +260,8 @@ __device__ __forceinline__ EMask<DT> code_step(uint32_t lut, uint4 v, int valid,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const uint32_t ws = w[k] << 1;  // exponents in bytes 1 and 3
-            const uint32_t c0 = lds_u8(lut + __byte_perm(ws, 0, 0x4441));
-            const uint32_t c1 = lds_u8(lut + (ws >> 24));
+            const uint32_t c0 = lds_u8(prmt(ws, lut, 0x7651u));
+            const uint32_t c1 = lds_u8(prmt(ws, lut, 0x7653u));
             cw += (c0 << (8 * k)) + (c1 << (8 * k + 4));
             // bytes 0 and 2: sign<<7 | mantissa of the two elements (bytes 1, 3 unused)
             x[k] = ((w[k] >> 8) & 0x00800080u) | (w[k] & 0xFF7FFF7Fu);
@@ -279,7 +287,7 @@ __device__ __forceinline__ EMask<DT> code_step(uint32_t lut, uint4 v, int valid,
         for (int k = 0; k < 4; ++k) {
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const uint32_t c = lds_u8(lut + ((w[k] >> (8 * b + 2)) & 0x1Fu));
+                const uint32_t c = lds_u8(prmt(w[k], lut, 0x7650u + uint32_t(b)));
                 cw[k >> 1] += c << (4 * (4 * (k & 1) + b));
             }
             if (STORE) {
@@ -329,6 +337,15 @@ __device__ __forceinline__ uint32_t exponent_at(uint4 v, uint32_t j) {
 template <int DT, typename Put>
 __device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &running, Put put) {
     const uint32_t c = popc_mask(m);
+    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+    if (any == 0) return;
+    if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+        // at most one escape per lane: its rank counts the lanes before it that have one
+        const uint32_t lane = threadIdx.x & 31;
+        if (c) put(running + __popc(any & ((1u << lane) - 1u)), exponent_at<DT>(v, first_bit(m) >> 2));
+        running += __popc(any);
+        return;
+    }
     uint32_t tot;
     const uint32_t prefix = warp_exclusive_prefix(c, &tot);
     if (tot) {
@@ -427,12 +444,15 @@ __device__ __forceinline__ void warp_load_plan(const EncodeParams<MAXB> &p, int 
         W.hdr[lane] = lane < 12 ? reinterpret_cast<const uint32_t *>(p.plans + 64 * size_t(t))[lane] : 0u;
     __syncwarp();
     const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
-    for (int e = lane; e < Dt<DT>::kBins; e += 32) {
+    const uint32_t lut = lut_addr(W);
+    for (int x = lane; x < 256; x += 32) {
+        // BF16: x is the exponent; E5M2: x is the element byte
+        const uint32_t e = (DT == SZ_BF16) ? uint32_t(x) : (uint32_t(x) >> 2) & 0x1Fu;
         uint32_t code = kEscape;
 #pragma unroll
         for (int c = 0; c < int(kCodes); ++c)
-            if (cb_byte(H.cbw, c) == uint32_t(e)) code = uint32_t(c);
-        W.lut[e] = uint8_t(code);
+            if (cb_byte(H.cbw, c) == e) code = uint32_t(c);
+        sts_u8(lut + uint32_t(x), code);
     }
     __syncwarp();
 }
@@ -483,7 +503,7 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
 
     using G = Geo<DT>;
     constexpr int QIT = G::IT / 4;  // steps per quarter block
-    const uint32_t lut = smem_u32(W.lut), stage = smem_u32(W.esc[slot]);
+    const uint32_t lut = lut_addr(W), stage = smem_u32(W.esc[slot]);
     const uint32_t nunits = 4u * uint32_t(nbk);
     uint32_t next_x = 0;
     for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) ring_issue<DT>(W, R, in, n, b0, next_x);
@@ -556,7 +576,7 @@ __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const Ch
         for (uint32_t x = lane; x < total; x += 32)
             if (dst + x < L.total) out[dst + x] = W.esc[slot][x];
     } else {
-        const uint32_t lut = smem_u32(W.lut);
+        const uint32_t lut = lut_addr(W);
 #pragma unroll 1
         for (int k = 0; k < g.nbk; ++k) {
             const uint64_t d = dst + W.blk_off[slot][k];
