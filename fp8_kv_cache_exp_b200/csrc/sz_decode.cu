@@ -260,18 +260,21 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
         // codes 0-7 from bytes 0-7, codes 8-15 from bytes 8-15 (selector with
         // the top bit flipped, so each half reads zero for the other's codes)
         const uint32_t x0 = f.c0 ^ 0x88888888u, x1 = f.c1 ^ 0x88888888u;
+        const uint32_t ev = f.b & 0x33333333u, od = f.b & 0xCCCCCCCCu;  // mantissas 0, 2 / 1, 3 of each byte
+        const uint32_t ahi = f.a >> 8;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const uint32_t cw = (k < 2) ? f.c0 : f.c1, cx = (k < 2) ? x0 : x1;
             const uint32_t sl = (k & 1) ? (cw >> 16) : cw, sh = (k & 1) ? (cx >> 16) : cx;
-            const uint32_t e4 = prmt(xt[0], xt[1], sl) | prmt(xt[2], xt[3], sh);
-            const uint32_t s4 = (f.a >> (4 * k)) & 0xFu;
-            const uint32_t sgn = (s4 * 0x10204080u) & 0x80808080u;
-            // 2-bit mantissas of the four elements (byte k of plane b) to bits 0-1 of each byte
-            const uint32_t m8 = prmt(f.b, 0u, 0x4440u + uint32_t(k));
-            const uint32_t t = (m8 | (m8 << 12)) & 0x000F000Fu;
-            const uint32_t mnt = (t | (t << 6)) & 0x03030303u;
-            o[k] = sgn | mnt | e4;
+            const uint32_t e_lo = prmt(xt[0], xt[1], sl), e_hi = prmt(xt[2], xt[3], sh);
+            // Spreads by multiplication (the partial products never overlap a
+            // kept bit): sign bits 4k..4k+3 of plane a to bit 7 of bytes 0-3,
+            // the four 2-bit mantissas of byte k of plane b to bits 0-1.
+            const uint32_t sa = (k < 2) ? f.a : ahi;
+            const uint32_t sg = (k & 1) ? (sa & 0xF0u) * 0x01020408u : (sa & 0x0Fu) * 0x10204080u;
+            const uint32_t mn = prmt(ev, 0u, 0x4440u + uint32_t(k)) * 0x1001u +
+                                prmt(od, 0u, 0x4440u + uint32_t(k)) * 0x40040u;
+            o[k] = ((sg & 0x80808080u) | e_hi) | ((mn & 0x03030303u) | e_lo);
         }
         m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
     }

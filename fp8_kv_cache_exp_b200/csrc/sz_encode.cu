@@ -291,8 +291,13 @@ __device__ __forceinline__ EMask<DT> code_step(uint32_t lut, uint4 v, int valid,
                 cw[k >> 1] += c << (4 * (4 * (k & 1) + b));
             }
             if (STORE) {
-                sign |= ((((w[k] >> 7) & 0x01010101u) * 0x01020408u) >> 24) << (4 * k);
-                mant |= (((w[k] & 0x03030303u) * 0x01041040u) >> 24) << (8 * k);
+                // gathers by multiplication (no two partial products share a
+                // bit): the four sign bits to bits 28-31, the four 2-bit
+                // mantissas to bits 24-31; then to their place in the planes
+                const uint32_t sg = (w[k] & 0x80808080u) * 0x00204081u;
+                const uint32_t mt = (w[k] & 0x03030303u) * 0x01041040u;
+                sign |= (sg >> (28 - 4 * k)) & (0xFu << (4 * k));
+                mant |= (mt >> (24 - 8 * k)) & (0xFFu << (8 * k));
             }
         }
         if (valid < 16) {
