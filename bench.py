@@ -211,17 +211,21 @@ def run_ours(args, rank, world, device):
     ws_g = [sz.new_workspace(dt, [wl.n[i] for i in g]) for g in groups] if args.mode != "batch" else [ws]
     plans_g = [plans[g[0]: g[-1] + 1] for g in groups]
 
+    # the buffers stay in place across steps: marshal each call's arrays once
+    batches = [sz.Batch(dt, [wl.xs[i] for i in g], [outs[i] for i in g], w, p, decs=[decs[i] for i in g])
+               for g, w, p in zip(groups, ws_g, plans_g)]
+
     def plan_all():
-        for g, w, p in zip(groups, ws_g, plans_g):
-            sz.sz_plan_batched(dt, [wl.xs[i] for i in g], w, p)
+        for b in batches:
+            b.plan()
 
     def encode_all():
-        for g, w, p in zip(groups, ws_g, plans_g):
-            sz.sz_encode_batched(dt, p, [wl.xs[i] for i in g], [outs[i] for i in g], w)
+        for b in batches:
+            b.encode()
 
     def decode_all():
-        for g, w in zip(groups, ws_g):
-            sz.sz_decode_batched(dt, [outs[i] for i in g], [decs[i] for i in g], w)
+        for b in batches:
+            b.decode()
 
     # correctness of this very configuration before timing
     plan_all(); encode_all(); decode_all()
@@ -333,12 +337,14 @@ def run_e2e(args, wl, device):
     outs = [torch.empty(sz.sz_max_compressed_size(dt, n), dtype=torch.uint8, device=device) for n in wl.n]
     stream = torch.cuda.current_stream()
 
+    batch = sz.Batch(dt, dev_in, outs, ws, plans, decs=dev_out)
+
     def step():
         for h, d in zip(host_in, dev_in):
             d.copy_(h, non_blocking=True)
-        sz.sz_plan_batched(dt, dev_in, ws, plans)
-        sz.sz_encode_batched(dt, plans, dev_in, outs, ws)
-        sz.sz_decode_batched(dt, outs, dev_out, ws)
+        batch.plan()
+        batch.encode()
+        batch.decode()
         for d, h in zip(dev_out, host_out):
             h.copy_(d, non_blocking=True)
 

@@ -18,7 +18,7 @@ __all__ = [
     "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
     "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched", "sz_decode",
     "sz_decode_batched", "sz_last_device_status", "sz_encode_noalloc", "dtype_of", "elem_bytes", "numel_of",
-    "new_workspace", "new_plans",
+    "new_workspace", "new_plans", "Batch",
 ]
 
 SZ_BF16 = 0
@@ -117,8 +117,16 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _ptr(x: torch.Tensor) -> int:
+    """Device address of a tensor's first element; the library reads and writes
+    its bytes as one contiguous run, so strided views are refused."""
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous (the codec addresses its bytes as one run)")
+    return x.data_ptr()
+
+
 def _p(x: torch.Tensor):
-    return ctypes.c_void_p(x.data_ptr())
+    return ctypes.c_void_p(_ptr(x))
 
 
 def _arr(ctype, values):
@@ -170,7 +178,7 @@ def sz_plan(dtype: int, x: torch.Tensor, ws: torch.Tensor, plan: torch.Tensor, s
 def sz_plan_batched(dtype: int, xs, ws: torch.Tensor, plans: torch.Tensor, stream=None):
     xs = list(xs)
     T = len(xs)
-    _check(lib.sz_plan_batched(dtype, T, _arr(ctypes.c_void_p, [x.data_ptr() for x in xs]),
+    _check(lib.sz_plan_batched(dtype, T, _arr(ctypes.c_void_p, [_ptr(x) for x in xs]),
                                _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs]),
                                _p(ws), ws.nbytes, _p(plans), _stream(stream)), "sz_plan_batched")
 
@@ -198,9 +206,9 @@ def sz_encode_batched(dtype: int, plans: torch.Tensor, xs, outs, ws: torch.Tenso
     xs, outs = list(xs), list(outs)
     T = len(xs)
     _check(lib.sz_encode_batched(
-        dtype, T, _p(plans), _arr(ctypes.c_void_p, [x.data_ptr() for x in xs]),
+        dtype, T, _p(plans), _arr(ctypes.c_void_p, [_ptr(x) for x in xs]),
         _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs]),
-        _arr(ctypes.c_void_p, [o.data_ptr() for o in outs]),
+        _arr(ctypes.c_void_p, [_ptr(o) for o in outs]),
         _arr(ctypes.c_size_t, [o.nbytes for o in outs]), _p(ws), ws.nbytes, _stream(stream)),
         "sz_encode_batched")
 
@@ -217,10 +225,58 @@ def sz_decode_batched(dtype: int, comps, outs, ws: torch.Tensor, comp_bytes=None
     T = len(comps)
     cbs = [c.nbytes for c in comps] if comp_bytes is None else [int(b) for b in comp_bytes]
     _check(lib.sz_decode_batched(
-        dtype, T, _arr(ctypes.c_void_p, [c.data_ptr() for c in comps]), _arr(ctypes.c_size_t, cbs),
-        _arr(ctypes.c_void_p, [o.data_ptr() for o in outs]),
+        dtype, T, _arr(ctypes.c_void_p, [_ptr(c) for c in comps]), _arr(ctypes.c_size_t, cbs),
+        _arr(ctypes.c_void_p, [_ptr(o) for o in outs]),
         _arr(ctypes.c_uint64, [numel_of(o, dtype) for o in outs]), _p(ws), ws.nbytes,
         _stream(stream)), "sz_decode_batched")
+
+
+class Batch:
+    """A fixed batch marshalled once for repeated batched calls.
+
+    The pointer and size arrays of sz_plan_batched / sz_encode_batched /
+    sz_decode_batched are built here; plan(), encode() and decode() pass them
+    straight to those C entry points.  For KV-cache buffers that stay in place
+    across steps this takes the per-call marshalling off the host.  The
+    tensors must stay alive and must not move while the Batch is in use.
+
+    xs: the raw tensors (encode input, decode output when decs is None);
+    outs: one stream buffer per tensor (encode output, decode input);
+    decs: decode outputs (default: xs); comp_bytes: bytes of each stream
+    that decode may read (default: the stream buffers' sizes).
+    """
+
+    def __init__(self, dtype: int, xs, outs, ws: torch.Tensor, plans: torch.Tensor, decs=None,
+                 comp_bytes=None):
+        xs, outs = list(xs), list(outs)
+        decs = xs if decs is None else list(decs)
+        if not (len(xs) == len(outs) == len(decs)) or not 1 <= len(xs) <= SZ_MAX_BATCH:
+            raise ValueError("xs, outs and decs must have the same length, 1..%d" % SZ_MAX_BATCH)
+        if plans.shape[0] < len(xs):
+            raise ValueError("one 64-byte plan per tensor")
+        self.dtype, self.T = int(dtype), len(xs)
+        self._keep = (xs, outs, decs, ws, plans)
+        self._in = _arr(ctypes.c_void_p, [_ptr(x) for x in xs])
+        self._n = _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs])
+        self._out = _arr(ctypes.c_void_p, [_ptr(o) for o in outs])
+        self._cap = _arr(ctypes.c_size_t, [o.nbytes for o in outs])
+        cbs = [o.nbytes for o in outs] if comp_bytes is None else [int(b) for b in comp_bytes]
+        self._cb = _arr(ctypes.c_size_t, cbs)
+        self._dec = _arr(ctypes.c_void_p, [_ptr(d) for d in decs])
+        self._dn = _arr(ctypes.c_uint64, [numel_of(d, dtype) for d in decs])
+        self._ws, self._wsb, self._plans = _p(ws), ws.nbytes, _p(plans)
+
+    def plan(self, stream=None):
+        _check(lib.sz_plan_batched(self.dtype, self.T, self._in, self._n, self._ws, self._wsb,
+                                   self._plans, _stream(stream)), "sz_plan_batched")
+
+    def encode(self, stream=None):
+        _check(lib.sz_encode_batched(self.dtype, self.T, self._plans, self._in, self._n, self._out,
+                                     self._cap, self._ws, self._wsb, _stream(stream)), "sz_encode_batched")
+
+    def decode(self, stream=None):
+        _check(lib.sz_decode_batched(self.dtype, self.T, self._out, self._cb, self._dec, self._dn,
+                                     self._ws, self._wsb, _stream(stream)), "sz_decode_batched")
 
 
 def sz_last_device_status(ws: torch.Tensor, stream=None) -> int:

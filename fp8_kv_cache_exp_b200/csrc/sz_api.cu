@@ -22,9 +22,13 @@ uint64_t total_tiles(int T, const uint64_t *n) {
 }
 
 int num_sms() {
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    sms = cache[dev].load(std::memory_order_acquire);
+    if (sms > 0) return sms;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(sms, std::memory_order_release);
     return sms;
 }
 

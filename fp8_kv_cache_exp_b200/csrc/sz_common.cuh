@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "splitzip.h"
 
 namespace sz {
@@ -40,6 +42,25 @@ enum : int {
 // histogram slot (plan leaves the histograms zero; decode zeroes its counters
 // before it returns), one 1 KB slot apart.
 constexpr uint32_t kClaimStride = 256;
+
+// Resident CTAs per SM of a kernel launched with `threads` threads and `smem`
+// bytes of dynamic shared memory, on the current device; the first call per
+// device also raises the kernel's dynamic shared-memory limit.  `cache` holds
+// one entry per device (a function-local static of the launcher).  0 on error.
+constexpr int kMaxDevices = 64;
+inline int resident_per_sm(const void *kern, int threads, size_t smem, std::atomic<int> *cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    const int known = cache[dev].load(std::memory_order_acquire);
+    if (known > 0) return known;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return 0;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
+        return 0;
+    cache[dev].store(per_sm, std::memory_order_release);
+    return per_sm;
+}
 
 __host__ __device__ constexpr uint64_t align256(uint64_t x) { return (x + 255u) & ~uint64_t(255); }
 __host__ __device__ constexpr uint64_t cdiv(uint64_t a, uint64_t b) { return (a + b - 1) / b; }

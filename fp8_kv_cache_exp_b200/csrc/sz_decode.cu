@@ -576,11 +576,9 @@ template <int DT, int MAXB>
 sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     auto kern = decode_kernel<DT, MAXB>;
     const size_t smem = sizeof(WarpSmem) * NW;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-        return SZ_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess || per_sm < 1)
-        return SZ_ERR_CUDA;
+    static std::atomic<int> cache[kMaxDevices];
+    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
+    if (per_sm < 1) return SZ_ERR_CUDA;
     DecodeParams<MAXB> p;
     p.ctl = a.ctl;
     p.claim = a.ctl + kCtlWords;  // the histogram slots

@@ -700,11 +700,9 @@ template <int DT, int MAXB>
 sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     auto kern = encode_kernel<DT, MAXB>;
     const size_t smem = sizeof(WarpShared) * NW;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-        return SZ_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess || per_sm < 1)
-        return SZ_ERR_CUDA;
+    static std::atomic<int> cache[kMaxDevices];
+    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
+    if (per_sm < 1) return SZ_ERR_CUDA;
     const uint64_t resident = uint64_t(a.num_sms) * per_sm;
     EncodeParams<MAXB> p;
     p.ctl = a.ctl;

@@ -271,13 +271,9 @@ sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
     p.total_items = p.item_begin[a.T];
     const size_t smem = size_t(C::kBins) * (NT / 2) * 4;
     auto kern = plan_kernel<DT, NT, MAXB>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return SZ_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem) != cudaSuccess ||
-        per_sm < 1)
-        return SZ_ERR_CUDA;
+    static std::atomic<int> cache[kMaxDevices];
+    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
+    if (per_sm < 1) return SZ_ERR_CUDA;
     uint64_t grid = uint64_t(a.num_sms) * per_sm;
     if (p.total_items < grid) grid = p.total_items;
     if (grid == 0) grid = 1;  // only empty tensors: block 0 writes their plans

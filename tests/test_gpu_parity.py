@@ -153,3 +153,30 @@ def test_batched_decode_claims_every_block_and_resets():
         plans2 = m.new_plans(len(xs))
         m.sz_plan_batched(dtype, xs, ws, plans2)
         assert torch.equal(plans2, plans)
+
+
+def test_prepared_batch_matches_functional_calls():
+    """Batch marshals the pointer arrays once; its calls give the same streams and
+    round trip as the per-call functions."""
+    m = sz()
+    rng = np.random.default_rng(33)
+    for dtype in (0, 1):
+        sizes = [4096 * 5 + 3, 0, 70000, 4096]
+        raws = [oracle_pins._kvlike(rng, n, dtype) for n in sizes]
+        xs = [from_raw(r, dtype) for r in raws]
+        ws = m.new_workspace(dtype, sizes)
+        plans = m.new_plans(len(xs))
+        outs = [torch.zeros(m.sz_max_compressed_size(dtype, n), dtype=torch.uint8, device="cuda") for n in sizes]
+        decs = [torch.full_like(x.view(torch.uint8), 0xA5).view(x.dtype) for x in xs]
+        b = m.Batch(dtype, xs, outs, ws, plans, decs=decs)
+        for _ in range(2):
+            b.plan()
+            b.encode()
+            b.decode()
+            assert m.sz_last_device_status(ws) == 0
+        totals = m.sz_compressed_sizes(plans)
+        for raw, out, tot, dec in zip(raws, outs, totals, decs):
+            assert np.array_equal(out[:tot].cpu().numpy(), oracle.encode(dtype, raw))
+            assert np.array_equal(dec.view(torch.uint8).cpu().numpy(), raw)
+    with pytest.raises(ValueError):
+        m.Batch(0, [torch.zeros(8, 8, dtype=torch.bfloat16, device="cuda").t()], [outs[0]], ws, plans)
