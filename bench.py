@@ -373,6 +373,18 @@ def run_e2e(args, wl, device):
 
 # ------------------------------------------------------- the oracle arm
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(cfg_name: str, budget_s: float):
     """Time the CPU oracle (as it stands) on one layer's K and V: plan + encode + decode."""
     import numpy as np
@@ -403,6 +415,7 @@ def oracle_sample(cfg_name: str, budget_s: float):
     raw_total = nbytes * reps
     return {
         "value": round(raw_total / (t_enc + t_dec) / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
         "sample": "%s layer 0 K+V (%.1f MB raw) x %d rep(s), single-threaded C oracle" % (cfg_name, nbytes / 1e6, reps),
         "encode_gbs": round(raw_total / t_enc / 1e9, 4), "decode_gbs": round(raw_total / t_dec / 1e9, 4),
         "seconds": round(t_enc + t_dec, 2),
