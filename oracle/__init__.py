@@ -53,6 +53,8 @@ class Oracle:
         L.orc_codebook.restype = ctypes.c_int
         L.orc_encode.argtypes = [ctypes.c_int, _u8p, ctypes.c_uint64, _u8p, ctypes.c_uint64]
         L.orc_encode.restype = ctypes.c_int64
+        L.orc_encode_codebook.argtypes = [ctypes.c_int, _u8p, ctypes.c_uint64, _u8p, _u8p, ctypes.c_uint64]
+        L.orc_encode_codebook.restype = ctypes.c_int64
         L.orc_decode.argtypes = [_u8p, ctypes.c_uint64, _u8p, ctypes.c_uint64]
         L.orc_decode.restype = ctypes.c_int
         self.lib = L
@@ -98,6 +100,26 @@ class Oracle:
             raise ValueError("orc_encode failed: %d" % -r)
         return out
 
+    def encode_codebook_status(self, dtype: int, x, cb, cap=None):
+        """Encode with the given 15-entry codebook; return (bytes written or -error, stream)."""
+        raw = _raw(x)
+        n = raw.size // elem_size(dtype)
+        cbv = np.ascontiguousarray(np.asarray(cb, dtype=np.uint8).reshape(-1))
+        if cbv.size != 15:
+            raise ValueError("a codebook has 15 entries")
+        if cap is None:
+            cap = self.compressed_size(dtype, n, n)
+        out = np.full(max(cap, 1), 0xA5, dtype=np.uint8)
+        r = int(self.lib.orc_encode_codebook(dtype, _u8(raw), n, _u8(cbv), _u8(out), cap))
+        return r, (out[:r].copy() if r >= 0 else out[:0])
+
+    def encode_codebook(self, dtype: int, x, cb) -> np.ndarray:
+        """Encode raw elements with a given codebook (codebook reuse); return the stream."""
+        r, out = self.encode_codebook_status(dtype, x, cb)
+        if r < 0:
+            raise ValueError("orc_encode_codebook failed: %d" % -r)
+        return out
+
     def decode_status(self, stream, n: int, dtype: int):
         """Decode; return (status, raw uint8 array)."""
         s = _raw(stream)
@@ -141,6 +163,14 @@ def encode(dtype, x):
 
 def encode_status(dtype, x, cap=None):
     return default().encode_status(dtype, x, cap)
+
+
+def encode_codebook(dtype, x, cb):
+    return default().encode_codebook(dtype, x, cb)
+
+
+def encode_codebook_status(dtype, x, cb, cap=None):
+    return default().encode_codebook_status(dtype, x, cb, cap)
 
 
 def decode(stream, n, dtype):

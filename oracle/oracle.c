@@ -206,20 +206,30 @@ static unsigned code_of(const uint8_t *cb, unsigned e)
     return ORC_ESCAPE;
 }
 
-/* Encode n elements into out (capacity cap bytes).
+/* Encode n elements into out (capacity cap bytes) with the codebook cb[15]
+ * given by the caller instead of the tensor's own.  Any 15 distinct exponent
+ * values of the dtype's range form a valid codebook, and the result is still
+ * lossless: exponents outside it take the escape path (SplitZip project page,
+ * Abstract: rare exponent values go through the sparse escape stream).  This
+ * is what lets a codebook found once be reused for other layers or later
+ * steps without a new histogram pass (the related-work list of the ZipServ
+ * page names exponent reuse across iterations: "CIERA: Cross-Iteration
+ * Exponent Reuse for Lossless Allgather in Sharded MoE Training").  The
+ * stream is an ordinary format-v1 stream: its header records cb and the
+ * escape count E that cb leaves.
  * Returns the stream length, or minus an ORC_ERR_* code. */
-int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint64_t cap)
+int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint8_t *cb,
+                            uint8_t *out, uint64_t cap)
 {
     if (dtype != ORC_BF16 && dtype != ORC_E5M2) return -ORC_ERR_DTYPE;
-    if ((n && !in) || !out || n >= (1ull << 32)) return -ORC_ERR_ARG;
+    if ((n && !in) || !out || !cb || n >= (1ull << 32)) return -ORC_ERR_ARG;
+    for (unsigned c = 0; c < ORC_CODES; c++) {
+        if (cb[c] >= exponent_values(dtype)) return -ORC_ERR_ARG;
+        for (unsigned d = 0; d < c; d++)
+            if (cb[d] == cb[c]) return -ORC_ERR_ARG;
+    }
 
-    /* 1. histogram and codebook */
-    uint64_t hist[256];
-    uint8_t cb[ORC_CODES];
-    orc_histogram(dtype, in, n, hist);
-    orc_codebook(dtype, hist, cb);
-
-    /* 2. escape count: every element whose exponent is not in the codebook */
+    /* 1. escape count: every element whose exponent is not in the codebook */
     uint64_t E = 0;
     for (uint64_t i = 0; i < n; i++)
         if (code_of(cb, exponent_of(dtype, element_bits(dtype, in, i))) == ORC_ESCAPE) E++;
@@ -228,7 +238,7 @@ int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint6
     if (cap < L.total) return -ORC_ERR_SMALL;
     memset(out, 0, L.total);
 
-    /* 3. header */
+    /* 2. header */
     put_u32(out + 0, ORC_MAGIC);
     put_u16(out + 4, ORC_VERSION);
     out[6] = (uint8_t)dtype;
@@ -239,7 +249,7 @@ int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint6
     out[39] = 0;
     put_u64(out + 40, L.total);
 
-    /* 4. one pass in element order: planes, codes, escapes, and the escape
+    /* 3. one pass in element order: planes, codes, escapes, and the escape
      *    count before each block (the exclusive prefix over blocks). */
     uint64_t k = 0;  /* escapes emitted so far */
     for (uint64_t i = 0; i < n; i++) {
@@ -262,6 +272,20 @@ int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint6
     }
     put_u32(out + 64 + 4 * L.nb, (uint32_t)k);  /* offsets[nb] = E */
     return (int64_t)L.total;
+}
+
+/* Encode n elements into out (capacity cap bytes) with the tensor's own
+ * codebook: its 15 most frequent exponent values (Abstract).
+ * Returns the stream length, or minus an ORC_ERR_* code. */
+int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint64_t cap)
+{
+    if (dtype != ORC_BF16 && dtype != ORC_E5M2) return -ORC_ERR_DTYPE;
+    if ((n && !in) || !out || n >= (1ull << 32)) return -ORC_ERR_ARG;
+    uint64_t hist[256];
+    uint8_t cb[ORC_CODES];
+    orc_histogram(dtype, in, n, hist);
+    orc_codebook(dtype, hist, cb);
+    return orc_encode_codebook(dtype, in, n, cb, out, cap);
 }
 
 /* Read and check a stream header.  On success fills dtype, n, E, cb and the

@@ -99,8 +99,9 @@ def expected_codebook(raw: np.ndarray, dtype: int) -> np.ndarray:
     return order[:15].astype(np.uint8)
 
 
-def check(stream, raw, dtype: int) -> None:
-    """Assert that `stream` is exactly the v1 encoding of `raw` (raises AssertionError)."""
+def check(stream, raw, dtype: int, codebook=None) -> None:
+    """Assert that `stream` is exactly the v1 encoding of `raw` (raises AssertionError):
+    with the tensor's own top-15 codebook, or with `codebook` when one is given."""
     s = np.asarray(stream, dtype=np.uint8)
     raw = np.asarray(raw, dtype=np.uint8).reshape(-1)
     n = raw.size // (2 if dtype == 0 else 1)
@@ -109,7 +110,7 @@ def check(stream, raw, dtype: int) -> None:
     assert f["version"] == 1 and f["dtype"] == dtype and f["block_log2"] == 12
     assert f["n"] == n
     assert f["pad"] == 0 and f["tail"] == bytes(16)
-    cb = expected_codebook(raw, dtype)
+    cb = expected_codebook(raw, dtype) if codebook is None else np.asarray(codebook, dtype=np.uint8)
     assert np.array_equal(f["cb"], cb), (f["cb"], cb)
     e = exponents(raw, dtype)
     lut = np.full(256, 15, dtype=np.uint8)

@@ -17,6 +17,10 @@ what:
                   exponents, uniform random bits (np.bincount + sort)
   ratio           ratio <= 16/12 (BF16) and <= 8/7 (E5M2): 12 and 7 coded bits
                   per element plus escapes (project page: "up to 1.14x" on FP8)
+  codebook reuse  encoding with a given codebook: the ordinary encoding when it
+                  is the tensor's own (found by numpy), the reader-checked v1
+                  encoding under any other, a hand-worked golden stream
+                  (bf16_n17_reuse.txt), and refusal of invalid codebooks
 """
 import itertools
 import os
@@ -24,6 +28,7 @@ import os
 import numpy as np
 
 import fieldcodec
+import oracle
 
 GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -31,7 +36,9 @@ GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 # ------------------------------------------------------------------ golden
 
 def load_golden(path):
-    """Parse a golden fixture: returns (dtype, raw input bytes, expected stream)."""
+    """Parse a golden fixture: returns (dtype, raw input bytes, expected stream).
+    A fixture with a `codebook` line was encoded with that given codebook; see
+    golden_codebook()."""
     dtype = n = total = None
     raw = None
     at = []
@@ -50,6 +57,8 @@ def load_golden(path):
             elif key == "input_hex":
                 words = [int(w, 16) for w in rest.split()]
                 raw = np.array(words, dtype="<u2" if dtype == 0 else np.uint8).view(np.uint8)
+            elif key == "codebook":
+                pass
             elif key == "at":
                 off, _, hexes = rest.partition(":")
                 at.append((int(off), bytes(int(h, 16) for h in hexes.split())))
@@ -60,6 +69,18 @@ def load_golden(path):
     return dtype, raw, expect
 
 
+def golden_codebook(path):
+    """The given codebook of a codebook-reuse fixture (15 uint8), or None."""
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line.startswith("codebook "):
+                cb = np.array([int(h, 16) for h in line.split()[1:]], dtype=np.uint8)
+                assert cb.size == 15
+                return cb
+    return None
+
+
 def golden_files():
     return sorted(os.path.join(GOLDEN_DIR, f) for f in os.listdir(GOLDEN_DIR) if f.endswith(".txt")
                   and f != "README.txt")
@@ -68,7 +89,8 @@ def golden_files():
 def pin_golden(orc):
     for path in golden_files():
         dtype, raw, expect = load_golden(path)
-        got = orc.encode(dtype, raw)
+        cb = golden_codebook(path)
+        got = orc.encode(dtype, raw) if cb is None else orc.encode_codebook(dtype, raw, cb)
         assert got.size == expect.size, (path, got.size, expect.size)
         diff = np.nonzero(got != expect)[0]
         assert diff.size == 0, (path, "first differing byte", int(diff[0]))
@@ -242,5 +264,44 @@ def pin_ratio_ceiling(orc):
         assert raw.size / orc.encode(dtype, raw).size > ceiling * 0.995
 
 
+# ---------------------------------------------------------- codebook reuse
+
+def pin_codebook_reuse(orc):
+    """Encoding with a given codebook: with the tensor's own codebook (found here
+    by numpy, not by the oracle) it is the ordinary encoding; with any other it is
+    still the v1 encoding of the data under that codebook, checked field by field
+    by the independent reader, and lossless; bad codebooks are refused."""
+    rng = np.random.default_rng(77)
+    for dtype in (0, 1):
+        nbins = 256 if dtype == 0 else 32
+        for n in (0, 1, 4095, 4096, 4097, 9000, 20000):
+            raw = _kvlike(rng, n, dtype)
+            own = fieldcodec.expected_codebook(raw, dtype)
+            assert np.array_equal(orc.encode_codebook(dtype, raw, own), orc.encode(dtype, raw))
+            other = _kvlike(rng, 5000, dtype)
+            foreign = [fieldcodec.expected_codebook(other, dtype),           # another tensor's
+                       rng.choice(nbins, 15, replace=False).astype(np.uint8),  # arbitrary
+                       np.arange(nbins - 15, nbins, dtype=np.uint8)]          # misses most values
+            for cb in foreign:
+                st = orc.encode_codebook(dtype, raw, cb)
+                fieldcodec.check(st, raw, dtype, codebook=cb)
+                assert np.array_equal(orc.decode(st, n, dtype), raw)
+        # nothing in the codebook occurs: every element escapes, E = n
+        raw = np.full(3000, 0x3F80 if dtype == 0 else 0x3C, dtype="<u2" if dtype == 0 else np.uint8).view(np.uint8)
+        e0 = int(fieldcodec.exponents(raw, dtype)[0])
+        cb = np.array([v for v in range(nbins) if v != e0][:15], dtype=np.uint8)
+        st = orc.encode_codebook(dtype, raw, cb)
+        assert fieldcodec.parse(st)["E"] == 3000
+        fieldcodec.check(st, raw, dtype, codebook=cb)
+        # refused: a repeated value, a value outside the exponent range
+        dup = cb.copy()
+        dup[3] = dup[2]
+        assert orc.encode_codebook_status(dtype, raw, dup)[0] == -oracle.ERR_ARG
+        if dtype == 1:  # every byte value is a BF16 exponent; 32 is out of E5M2's range
+            big = cb.copy()
+            big[0] = 32
+            assert orc.encode_codebook_status(dtype, raw, big)[0] == -oracle.ERR_ARG
+
+
 ALL_PINS = (pin_golden, pin_exhaustive_bf16, pin_exhaustive_e5m2, pin_ragged_sizes,
-            pin_bruteforce_codebook, pin_special_cases, pin_ratio_ceiling)
+            pin_bruteforce_codebook, pin_special_cases, pin_ratio_ceiling, pin_codebook_reuse)

@@ -48,6 +48,11 @@ MUTANTS = {
                           ("if (get_u32(comp + 64 + 4 * L.nb) != E) return ORC_ERR_CORRUPT;", "", 1)],
     "escape_counter_not_advanced": [("            k++;\n        }\n    }\n    put_u32", "        }\n    }\n    put_u32", 1)],
     "table_one_entry_short": [("64u + 4u * (L.nb + 1u)", "64u + 4u * L.nb", 1)],
+    "given_codebook_duplicates_accepted": [("if (cb[d] == cb[c]) return -ORC_ERR_ARG;", "(void)d;", 1)],
+    "given_codebook_replaced_by_own": [
+        ("    /* 1. escape count: every element whose exponent is not in the codebook */",
+         "    uint64_t own_h[256];\n    uint8_t own_cb[ORC_CODES];\n"
+         "    orc_histogram(dtype, in, n, own_h);\n    orc_codebook(dtype, own_h, own_cb);\n    cb = own_cb;", 1)],
 }
 
 
