@@ -16,7 +16,8 @@ __all__ = [
     "SZ_BF16", "SZ_FP8_E5M2", "SZ_OK", "SplitZipError", "lib", "lib_path",
     "sz_status_string", "sz_workspace_bytes", "sz_workspace_bytes_batched", "sz_stream_bytes",
     "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
-    "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched", "sz_decode",
+    "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched",
+    "sz_encode_reuse", "sz_encode_reuse_batched", "sz_decode",
     "sz_decode_batched", "sz_last_device_status", "sz_encode_noalloc", "dtype_of", "elem_bytes", "numel_of",
     "new_workspace", "new_plans", "Batch",
 ]
@@ -62,6 +63,8 @@ def _load():
         "sz_compressed_sizes": (i32, [i32, vp, pu64, vp]),
         "sz_encode": (i32, [i32, vp, vp, u64, vp, sz, vp, sz, vp]),
         "sz_encode_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, sz, vp]),
+        "sz_encode_reuse": (i32, [i32, vp, vp, u64, vp, sz, vp, vp, sz, vp]),
+        "sz_encode_reuse_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, vp, sz, vp]),
         "sz_decode": (i32, [i32, vp, sz, vp, u64, vp, sz, vp]),
         "sz_decode_batched": (i32, [i32, i32, pvp, psz, pvp, pu64, vp, sz, vp]),
         "sz_last_device_status": (i32, [vp, vp]),
@@ -213,6 +216,32 @@ def sz_encode_batched(dtype: int, plans: torch.Tensor, xs, outs, ws: torch.Tenso
         "sz_encode_batched")
 
 
+def _opt(t):
+    return None if t is None else _p(t)
+
+
+def sz_encode_reuse(dtype: int, codebook: torch.Tensor, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+                    total: torch.Tensor = None, stream=None):
+    """Encode with the codebook of an earlier plan (codebook reuse); `total`, if
+    given, is a device int64 tensor that receives the stream's length."""
+    _check(lib.sz_encode_reuse(dtype, _p(codebook), _p(x), numel_of(x, dtype), _p(out), out.nbytes, _opt(total),
+                               _p(ws), ws.nbytes, _stream(stream)), "sz_encode_reuse")
+
+
+def sz_encode_reuse_batched(dtype: int, codebooks: torch.Tensor, xs, outs, ws: torch.Tensor,
+                            totals: torch.Tensor = None, stream=None):
+    """Codebook reuse for a batch: tensor t uses the codebook of plan t of `codebooks`;
+    `totals`, if given, is a device int64 tensor of T stream lengths."""
+    xs, outs = list(xs), list(outs)
+    T = len(xs)
+    _check(lib.sz_encode_reuse_batched(
+        dtype, T, _p(codebooks), _arr(ctypes.c_void_p, [_ptr(x) for x in xs]),
+        _arr(ctypes.c_uint64, [numel_of(x, dtype) for x in xs]),
+        _arr(ctypes.c_void_p, [_ptr(o) for o in outs]),
+        _arr(ctypes.c_size_t, [o.nbytes for o in outs]), _opt(totals), _p(ws), ws.nbytes, _stream(stream)),
+        "sz_encode_reuse_batched")
+
+
 def sz_decode(dtype: int, comp: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, comp_bytes=None,
               stream=None):
     cb = comp.nbytes if comp_bytes is None else int(comp_bytes)
@@ -273,6 +302,16 @@ class Batch:
     def encode(self, stream=None):
         _check(lib.sz_encode_batched(self.dtype, self.T, self._plans, self._in, self._n, self._out,
                                      self._cap, self._ws, self._wsb, _stream(stream)), "sz_encode_batched")
+
+    def encode_reuse(self, codebooks: torch.Tensor = None, totals: torch.Tensor = None, stream=None):
+        """Encode with reused codebooks: plan t of `codebooks` (default: this batch's
+        plans, as left by an earlier plan()) for tensor t, no histogram pass."""
+        cbs = self._plans if codebooks is None else _p(codebooks)
+        if codebooks is not None:
+            self._keep_cb = codebooks
+        _check(lib.sz_encode_reuse_batched(self.dtype, self.T, cbs, self._in, self._n, self._out, self._cap,
+                                           _opt(totals), self._ws, self._wsb, _stream(stream)),
+               "sz_encode_reuse_batched")
 
     def decode(self, stream=None):
         _check(lib.sz_decode_batched(self.dtype, self.T, self._out, self._cb, self._dec, self._dn,

@@ -129,13 +129,17 @@ sz_status sz_compressed_size(const sz_plan_t *d_plan, uint64_t *h_bytes, cudaStr
     return sz_compressed_sizes(1, d_plan, h_bytes, stream);
 }
 
-sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
-                            const void *const *d_in, const uint64_t *n, void *const *d_out,
-                            const size_t *out_cap, void *d_ws, size_t ws_bytes,
-                            cudaStream_t stream) {
+namespace {
+
+// Ordinary encode (plans are the tensors' own) or codebook reuse (plans give
+// codebooks only).
+sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
+                        const uint64_t *n, void *const *d_out, const size_t *out_cap, uint64_t *d_totals,
+                        bool reuse, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
     sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
     if (s != SZ_OK) return s;
     if (!d_plans || !aligned(d_plans, 8) || !d_in || !d_out || !out_cap) return SZ_ERR_INVALID_ARG;
+    if (d_totals && !aligned(d_totals, 8)) return SZ_ERR_INVALID_ARG;
     for (int t = 0; t < T; ++t) {
         if (n[t] && (!d_in[t] || !aligned(d_in[t], 16))) return SZ_ERR_INVALID_ARG;
         if (!d_out[t] || !aligned(d_out[t], 16)) return SZ_ERR_INVALID_ARG;
@@ -156,7 +160,18 @@ sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
     a.cap = out_cap;
     a.ctl = reinterpret_cast<uint32_t *>(ws);
     a.status = reinterpret_cast<unsigned long long *>(ws + w.status);
+    a.totals = reinterpret_cast<unsigned long long *>(d_totals);
+    a.reuse = reuse ? 1 : 0;
     return launch_encode(a, stream);
+}
+
+}  // namespace
+
+sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
+                            const void *const *d_in, const uint64_t *n, void *const *d_out,
+                            const size_t *out_cap, void *d_ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+    return encode_common(dtype, T, d_plans, d_in, n, d_out, out_cap, nullptr, false, d_ws, ws_bytes, stream);
 }
 
 sz_status sz_encode(sz_dtype dtype, const sz_plan_t *d_plan, const void *d_in, uint64_t n,
@@ -164,6 +179,23 @@ sz_status sz_encode(sz_dtype dtype, const sz_plan_t *d_plan, const void *d_in, u
     const void *in[1] = {d_in};
     void *out[1] = {d_out};
     return sz_encode_batched(dtype, 1, d_plan, in, &n, out, &out_cap, d_ws, ws_bytes, stream);
+}
+
+sz_status sz_encode_reuse_batched(sz_dtype dtype, int T, const sz_plan_t *d_codebooks,
+                                  const void *const *d_in, const uint64_t *n, void *const *d_out,
+                                  const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    return encode_common(dtype, T, d_codebooks, d_in, n, d_out, out_cap, d_totals, true, d_ws, ws_bytes,
+                         stream);
+}
+
+sz_status sz_encode_reuse(sz_dtype dtype, const sz_plan_t *d_codebook, const void *d_in, uint64_t n,
+                          void *d_out, size_t out_cap, uint64_t *d_total, void *d_ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+    const void *in[1] = {d_in};
+    void *out[1] = {d_out};
+    return sz_encode_reuse_batched(dtype, 1, d_codebook, in, &n, out, &out_cap, d_total, d_ws, ws_bytes,
+                                   stream);
 }
 
 sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,

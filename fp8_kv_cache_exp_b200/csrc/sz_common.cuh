@@ -156,6 +156,8 @@ struct EncodeParams {
     uint32_t *ctl;
     unsigned long long *status;  // one look-back word per global chunk
     const uint8_t *plans;
+    unsigned long long *totals;  // per-tensor stream bytes out (may be null)
+    int reuse;                   // plans give codebooks only: E and the total are found here
     uint32_t total_chunks;
     uint32_t total_jobs;         // chunks + empty tensors
     int T;

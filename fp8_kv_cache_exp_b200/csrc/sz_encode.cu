@@ -143,11 +143,41 @@ __device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t 
     return true;
 }
 
+// The plan's codebook: 15 distinct values inside the exponent range and a zero
+// pad byte (one lane per entry; warp-wide).
 template <int DT>
-__device__ __forceinline__ bool header_ok(const Header &H, uint64_t n, uint64_t cap,
-                                          uint32_t *why) {
-    if (H.magic != kMagic || H.vtag != header_vtag(DT) || H.n != n || H.E > n ||
-        (H.cbw[3] >> 24) != 0 || H.total != stream_layout(DT, n, H.E).total) {
+__device__ __forceinline__ bool codebook_ok(const Header &H) {
+    const int lane = threadIdx.x & 31;
+    bool ok = (H.cbw[3] >> 24) == 0;
+    if (lane < int(kCodes)) {
+        const uint32_t v = cb_byte(H.cbw, lane);
+        ok = ok && v < uint32_t(Dt<DT>::kBins);
+        for (int d = 0; d < lane; ++d) ok = ok && cb_byte(H.cbw, d) != v;
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Check a tensor's plan before coding it (warp-wide).  Ordinary encode: the
+// plan is this tensor's header (n, E, codebook, total) and its total must fit
+// the output.  Codebook reuse: only the codebook is taken from the plan; the
+// smallest stream for n must fit (escapes are bounded by the capacity later).
+template <int DT>
+__device__ __forceinline__ bool plan_ok(const Header &H, uint64_t n, uint64_t cap, bool reuse,
+                                        uint32_t *why) {
+    const bool cb = codebook_ok<DT>(H);
+    if (reuse) {
+        if (!cb) {
+            *why = SZ_ERR_PLAN_MISMATCH;
+            return false;
+        }
+        if (stream_layout(DT, n, 0).total > cap) {
+            *why = SZ_ERR_BUFFER_TOO_SMALL;
+            return false;
+        }
+        return true;
+    }
+    if (!cb || H.magic != kMagic || H.vtag != header_vtag(DT) || H.n != n || H.E > n ||
+        H.total != stream_layout(DT, n, H.E).total) {
         *why = SZ_ERR_PLAN_MISMATCH;
         return false;
     }
@@ -158,14 +188,33 @@ __device__ __forceinline__ bool header_ok(const Header &H, uint64_t n, uint64_t 
     return true;
 }
 
+// Word `lane` (< 16) of the 64-byte stream header for n elements, E escapes
+// and codebook words cbw.
+template <int DT>
+__device__ __forceinline__ uint32_t header_word(int lane, uint64_t n, uint64_t E, uint64_t total,
+                                                const uint32_t (&cbw)[4]) {
+    uint32_t w = 0;
+    w = lane == 0 ? kMagic : w;
+    w = lane == 1 ? header_vtag(DT) : w;
+    w = lane == 2 ? uint32_t(n) : w;
+    w = lane == 3 ? uint32_t(n >> 32) : w;
+    w = lane == 4 ? uint32_t(E) : w;
+    w = lane == 5 ? uint32_t(E >> 32) : w;
+    w = (lane >= 6 && lane < 10) ? pick4(cbw[0], cbw[1], cbw[2], cbw[3], uint32_t(lane - 6)) : w;
+    w = lane == 10 ? uint32_t(total) : w;
+    w = lane == 11 ? uint32_t(total >> 32) : w;
+    return w;
+}
+
 __device__ __forceinline__ void zero_bytes(uint8_t *out, uint64_t a, uint64_t b) {
     for (uint64_t x = a + (threadIdx.x & 31); x < b; x += 32) out[x] = 0;
 }
 
-// Header, offsets[nb] and the zero gaps between sections (once per stream, one warp).
-__device__ void write_stream_frame(uint8_t *out, const Layout &L, const uint32_t *hdr, uint64_t E) {
+// Header (lane l < 16 holds word l), offsets[nb] and the zero gaps between
+// sections (once per stream, one warp).
+__device__ void write_stream_frame(uint8_t *out, const Layout &L, uint32_t hdr_word, uint64_t E) {
     const int lane = threadIdx.x & 31;
-    if (lane < 16) reinterpret_cast<uint32_t *>(out)[lane] = hdr[lane];
+    if (lane < 16) reinterpret_cast<uint32_t *>(out)[lane] = hdr_word;
     if (lane == 0) *reinterpret_cast<uint32_t *>(out + 64 + 4 * L.nb) = uint32_t(E);
     zero_bytes(out, L.tab_end, L.plane[0]);
 #pragma unroll
@@ -500,11 +549,11 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
     }
     const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     uint32_t why = 0;
-    if (!header_ok<DT>(H, n, p.cap[g.t], &why)) {
+    if (!plan_ok<DT>(H, n, p.cap[g.t], p.reuse != 0, &why)) {
         if (lane == 0 && g.chunk == 0) set_error(p.ctl, why, uint32_t(g.t));
         return 0xFFFFFFFFu;  // every chunk of this tensor takes this branch: no look-back waits on it
     }
-    const Layout L = stream_layout(DT, n, H.E);
+    const Layout L = stream_layout(DT, n, p.reuse ? 0 : H.E);  // section starts do not depend on E
 
     using G = Geo<DT>;
     constexpr int QIT = G::IT / 4;  // steps per quarter block
@@ -565,32 +614,44 @@ template <int DT, int MAXB>
 __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
                              uint32_t total, const Lookback &lb, WarpShared &W) {
     const int lane = threadIdx.x & 31;
-    const uint8_t *hdr = p.plans + 64 * size_t(g.t);
-    const Header H = load_header(hdr);
-    const Layout L = stream_layout(DT, g.n, H.E);
+    const Header H = load_header(p.plans + 64 * size_t(g.t));
+    const bool reuse = p.reuse != 0;
+    const Layout L = stream_layout(DT, g.n, reuse ? 0 : H.E);
     uint8_t *out = p.out[g.t];
     const uint32_t excl = lb.excl;
+    const bool last = g.b0 + g.nbk == g.nb;
     if (lane == 0) {
         if (lb.flags & kLbTimedOut) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
-        if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-        if (g.b0 + g.nbk == g.nb && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+        if (!reuse) {
+            if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+            if (last && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+        }
     }
     if (lane < g.nbk) *reinterpret_cast<uint32_t *>(out + 64 + 4 * (g.b0 + lane)) = excl + W.blk_off[slot][lane];
+    // escapes past the stream's end (ordinary encode) or the buffer's (reuse) are not written
+    const uint64_t bound = reuse ? p.cap[g.t] : L.total;
     const uint64_t dst = L.esc + excl;
     if (total <= kWarpStage) {
         for (uint32_t x = lane; x < total; x += 32)
-            if (dst + x < L.total) out[dst + x] = W.esc[slot][x];
+            if (dst + x < bound) out[dst + x] = W.esc[slot][x];
     } else {
         const uint32_t lut = lut_addr(W);
 #pragma unroll 1
         for (int k = 0; k < g.nbk; ++k) {
             const uint64_t d = dst + W.blk_off[slot][k];
             code_block<DT, false>(lut, p.in[g.t], g.n, g.b0 + k, L, out, [&](uint32_t r, uint32_t e) {
-                if (d + r < L.total) out[d + r] = uint8_t(e);
+                if (d + r < bound) out[d + r] = uint8_t(e);
             });
         }
     }
-    if (g.b0 + g.nbk == g.nb) write_stream_frame(out, L, reinterpret_cast<const uint32_t *>(hdr), H.E);
+    if (last) {
+        // the tensor's escape count is now known: excl + total
+        const uint64_t E = reuse ? uint64_t(excl) + total : H.E;
+        const uint64_t stream_total = stream_layout(DT, g.n, E).total;
+        if (reuse && stream_total > p.cap[g.t] && lane == 0) set_error(p.ctl, SZ_ERR_BUFFER_TOO_SMALL, job);
+        write_stream_frame(out, L, header_word<DT>(lane, g.n, E, stream_total, H.cbw), E);
+        if (p.totals && lane == 0) p.totals[g.t] = stream_total;
+    }
     __syncwarp();
 }
 
@@ -602,11 +663,13 @@ __device__ void encode_empty(const EncodeParams<MAXB> &p, int t, WarpShared &W, 
     plan_tensor = t;
     const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     uint32_t why = 0;
-    if (!header_ok<DT>(H, 0, p.cap[t], &why)) {
+    if (!plan_ok<DT>(H, 0, p.cap[t], p.reuse != 0, &why)) {
         if (lane == 0) set_error(p.ctl, why, uint32_t(t));
         return;
     }
-    write_stream_frame(p.out[t], stream_layout(DT, 0, 0), W.hdr, 0);
+    const Layout L = stream_layout(DT, 0, 0);
+    write_stream_frame(p.out[t], L, header_word<DT>(lane, 0, 0, L.total, H.cbw), 0);
+    if (p.totals && lane == 0) p.totals[t] = L.total;
 }
 
 // A chunk whose offset is still being looked up.
@@ -708,6 +771,8 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     p.ctl = a.ctl;
     p.status = a.status;
     p.plans = a.plans;
+    p.totals = a.totals;
+    p.reuse = a.reuse;
     p.T = a.T;
     p.n_empty = 0;
     p.chunk_log2 = 3;  // kChunkBlocks

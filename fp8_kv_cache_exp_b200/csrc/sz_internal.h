@@ -26,6 +26,8 @@ struct EncodeArgs {
     const size_t *cap;
     uint32_t *ctl;
     unsigned long long *status;
+    unsigned long long *totals;  // may be null
+    int reuse;                   // codebook reuse: plans give codebooks only
 };
 
 struct DecodeArgs {

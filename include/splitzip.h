@@ -154,6 +154,38 @@ sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
                             const size_t *out_cap, void *d_ws, size_t ws_bytes,
                             cudaStream_t stream);
 
+/* Codebook reuse: encode with the codebook of a plan made earlier -- for
+ * another layer, or for the same tensor at an earlier step -- without a new
+ * histogram pass.  Any codebook keeps the stream lossless: every exponent
+ * outside it is escaped (project page, Abstract: rare exponent values go
+ * through the sparse escape stream).  The stream is an ordinary format-v1
+ * stream that sz_decode reads; its header records the given codebook and the
+ * escape count E that codebook leaves for this data.
+ *
+ * Only the codebook bytes (plan bytes 24..39, 15 distinct values of the
+ * dtype's exponent range, byte 39 zero) are read from d_codebook; its n, E
+ * and total are ignored.  An invalid codebook is reported as
+ * SZ_ERR_PLAN_MISMATCH on the device error word and nothing is written.
+ *
+ * out_cap must hold at least sz_stream_bytes(dtype, n, 0) (checked here).
+ * The total is known only when the last block is coded: if the escapes do not
+ * fit, SZ_ERR_BUFFER_TOO_SMALL is recorded and the stream is incomplete
+ * (sz_max_compressed_size always suffices).  d_total (device, 8-byte aligned,
+ * or NULL) receives the stream's length; the header holds it too (bytes
+ * 40..47). */
+sz_status sz_encode_reuse(sz_dtype dtype, const sz_plan_t *d_codebook, const void *d_in, uint64_t n,
+                          void *d_out, size_t out_cap, uint64_t *d_total, void *d_ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/* Codebook reuse for T tensors in one launch.  d_in, n, d_out, out_cap are
+ * HOST arrays of T entries; d_codebooks are T consecutive plans in device
+ * memory (tensor t uses the codebook of plan t); d_totals (device, or NULL)
+ * receives T stream lengths. */
+sz_status sz_encode_reuse_batched(sz_dtype dtype, int T, const sz_plan_t *d_codebooks,
+                                  const void *const *d_in, const uint64_t *n, void *const *d_out,
+                                  const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+
 /* Decode a stream of comp_bytes bytes holding n elements of dtype into d_out
  * (BF16: 2n bytes, E5M2: n bytes); the result is bitwise identical to the
  * encoded input (project page, FAQ "Is SplitZip lossy?").  A stream that fails

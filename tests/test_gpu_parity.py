@@ -66,9 +66,22 @@ def test_special_cases():
 
 
 def test_golden_streams_on_gpu():
+    m = sz()
     for path in oracle_pins.golden_files():
         dtype, raw, expect = oracle_pins.load_golden(path)
-        plan, stream = gpu_encode(dtype, from_raw(raw, dtype))
+        cb = oracle_pins.golden_codebook(path)
+        if cb is None:
+            plan, stream = gpu_encode(dtype, from_raw(raw, dtype))
+        else:  # a codebook-reuse fixture: encode with the given codebook
+            x = from_raw(raw, dtype)
+            n = m.numel_of(x, dtype)
+            ws = m.new_workspace(dtype, [n])
+            h = np.zeros((1, 64), dtype=np.uint8)
+            h[0, 24:39] = cb
+            out = torch.full((m.sz_max_compressed_size(dtype, n),), 0xA5, dtype=torch.uint8, device="cuda")
+            m.sz_encode_reuse(dtype, torch.from_numpy(h).cuda(), x, out, ws)
+            assert m.sz_last_device_status(ws) == 0
+            stream = out[: expect.size].cpu().numpy()
         assert np.array_equal(stream, expect), path
         n = raw.size // (2 if dtype == 0 else 1)
         assert np.array_equal(gpu_decode(dtype, expect, n), raw), path
