@@ -192,6 +192,36 @@ class Workload:
         self.raw_bytes = sum(self.n) * self.esize
 
 
+def paged_pools(wl, page_tokens: int, device):
+    """Two page pools holding the workload's tensors in pages of page_tokens
+    tokens, each in its own random page order (seeded).  Returns (source pool,
+    destination pool, source page tables, destination page tables, elements per page)."""
+    shape = wl.xs[0].shape  # [tokens, heads, head_dim]
+    page_elems = page_tokens * shape[1] * shape[2]
+    if page_elems % 1024:
+        raise SystemExit("--paged: a page must hold a multiple of 1024 elements")
+    counts = [-(-n // page_elems) for n in wl.n]
+    total = sum(counts)
+    pb = page_elems * wl.esize
+    src_pool = torch.empty(total * pb, dtype=torch.uint8, device=device)
+    dst_pool = torch.zeros(total * pb, dtype=torch.uint8, device=device)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(7_000_000 + page_tokens)
+    src_order = torch.randperm(total, generator=g).to(torch.int32)
+    dst_order = torch.randperm(total, generator=g).to(torch.int32)
+    src_tabs, dst_tabs, k = [], [], 0
+    for x, c in zip(wl.xs, counts):
+        sid, did = src_order[k: k + c].to(device), dst_order[k: k + c].to(device)
+        k += c
+        flat = x.view(torch.uint8).reshape(-1)
+        padded = torch.zeros(c * pb, dtype=torch.uint8, device=device)
+        padded[: flat.numel()] = flat
+        src_pool.view(total, pb)[sid.long()] = padded.view(c, pb)
+        src_tabs.append(sid)
+        dst_tabs.append(did)
+    return src_pool, dst_pool, src_tabs, dst_tabs, page_elems
+
+
 def run_ours(args, rank, world, device):
     import fp8_kv_cache_exp_b200 as sz
     wl = Workload(args.workload, rank, world, device, args.layers)
@@ -212,8 +242,19 @@ def run_ours(args, rank, world, device):
     plans_g = [plans[g[0]: g[-1] + 1] for g in groups]
 
     # the buffers stay in place across steps: marshal each call's arrays once
-    batches = [sz.Batch(dt, [wl.xs[i] for i in g], [outs[i] for i in g], w, p, decs=[decs[i] for i in g])
-               for g, w, p in zip(groups, ws_g, plans_g)]
+    if args.paged:
+        # paged KV: every tensor's pages sit in one pool in a random order (the
+        # prefill side), and decode writes into a second pool with its own random
+        # page order (the decode side)
+        src_pool, dst_pool, src_tabs, dst_tabs, page_elems = paged_pools(wl, args.paged, device)
+        srcs = [sz.paged(dt, src_pool, tb, page_elems) for tb in src_tabs]
+        dsts = [sz.paged(dt, dst_pool, tb, page_elems) for tb in dst_tabs]
+        batches = [sz.Batch(dt, None, [outs[i] for i in g], w, p, src_pages=[srcs[i] for i in g],
+                            dst_pages=[dsts[i] for i in g], n=[wl.n[i] for i in g])
+                   for g, w, p in zip(groups, ws_g, plans_g)]
+    else:
+        batches = [sz.Batch(dt, [wl.xs[i] for i in g], [outs[i] for i in g], w, p, decs=[decs[i] for i in g])
+                   for g, w, p in zip(groups, ws_g, plans_g)]
 
     def plan_all():
         for b in batches:
@@ -237,8 +278,11 @@ def run_ours(args, rank, world, device):
         st = sz.sz_last_device_status(w)
         if st != 0:
             raise RuntimeError("device status %s" % sz.sz_status_string(st))
+    if args.paged:
+        decs = [dst_pool.view(-1, page_elems * wl.esize)[tb.long()].reshape(-1)[: n * wl.esize]
+                for tb, n in zip(dst_tabs, wl.n)]
     for x, d in zip(wl.xs, decs):
-        if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
+        if not torch.equal(x.view(torch.uint8).reshape(-1), d.view(torch.uint8).reshape(-1)):
             raise RuntimeError("round trip mismatch")
     totals = sz.sz_compressed_sizes(plans)
     stream_bytes = sum(totals)
@@ -318,6 +362,8 @@ def run_ours(args, rank, world, device):
         "config": {"workload": wl.name, "desc": wl.desc, "tensors_per_rank": T,
                    "codebooks": "reused from a calibration plan (no histogram pass per step)" if args.reuse
                    else "own plan per step",
+                   "layout": ("paged: %d-token pages, random page order in and out" % args.paged) if args.paged
+                   else "contiguous tensors",
                    "raw_bytes_per_rank": wl.raw_bytes, "mode": "one batch" if args.mode == "batch" else "per layer",
                    "l2": "inputs larger than L2 (%.2f GB per step per rank)" % (wl.raw_bytes / 1e9),
                    "parallelism": "replicas" if world == 1 else "dp%d (independent tensors)" % world},
@@ -484,6 +530,8 @@ def main():
                     help="layers per step (default: the workload's); smaller batches are for profiler captures")
     ap.add_argument("--reuse", action="store_true",
                     help="codebook reuse: plan once, then every step is encode with those codebooks + decode")
+    ap.add_argument("--paged", type=int, default=0, metavar="TOKENS",
+                    help="hold the tensors in pages of TOKENS tokens (paged KV), in random page order")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -507,7 +555,7 @@ def main():
                                 device_id=device)
     try:
         res, wl = run_ours(args, rank, world, device)
-        if not args.no_e2e:
+        if not args.no_e2e and not args.paged:  # e2e covers the contiguous path
             e2e = run_e2e(args, wl, device)
             e2e_val = sum_over_ranks(wl.raw_bytes, world, device) / (
                 max_over_ranks(e2e["ms_per_step"], world, device) * 1e-3) / 1e9

@@ -17,7 +17,8 @@ __all__ = [
     "sz_status_string", "sz_workspace_bytes", "sz_workspace_bytes_batched", "sz_stream_bytes",
     "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
     "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched",
-    "sz_encode_reuse", "sz_encode_reuse_batched", "sz_decode",
+    "sz_encode_reuse", "sz_encode_reuse_batched", "sz_plan_paged_batched", "sz_encode_paged_batched",
+    "sz_decode_paged_batched", "sz_encode_reuse_paged_batched", "sz_paged_t", "paged", "sz_decode",
     "sz_decode_batched", "sz_last_device_status", "sz_encode_noalloc", "dtype_of", "elem_bytes", "numel_of",
     "new_workspace", "new_plans", "Batch",
 ]
@@ -43,6 +44,12 @@ SZ_NOALLOC_MAX_ELEMS = 1 << 27
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitzip.so")
 
 
+class sz_paged_t(ctypes.Structure):
+    """C layout of sz_paged_t (include/splitzip.h): a tensor held in pages of a pool."""
+    _fields_ = [("pool", ctypes.c_void_p), ("pages", ctypes.c_void_p), ("pool_pages", ctypes.c_uint64),
+                ("page_bytes", ctypes.c_uint64), ("page_elems", ctypes.c_uint32)]
+
+
 def _load():
     if not os.path.exists(lib_path):
         raise ImportError("libsplitzip.so is not built (%s); run: python fp8_kv_cache_exp_b200/build.py"
@@ -50,6 +57,7 @@ def _load():
     L = ctypes.CDLL(lib_path)
     vp, u64, sz, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_int
     pvp, pu64, psz = ctypes.POINTER(vp), ctypes.POINTER(u64), ctypes.POINTER(sz)
+    ppg = ctypes.POINTER(sz_paged_t)
     sigs = {
         "sz_status_string": (ctypes.c_char_p, [i32]),
         "sz_workspace_bytes": (sz, [i32, u64]),
@@ -65,6 +73,10 @@ def _load():
         "sz_encode_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, sz, vp]),
         "sz_encode_reuse": (i32, [i32, vp, vp, u64, vp, sz, vp, vp, sz, vp]),
         "sz_encode_reuse_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, vp, sz, vp]),
+        "sz_plan_paged_batched": (i32, [i32, i32, ppg, pu64, vp, sz, vp, vp]),
+        "sz_encode_paged_batched": (i32, [i32, i32, vp, ppg, pu64, pvp, psz, vp, sz, vp]),
+        "sz_decode_paged_batched": (i32, [i32, i32, pvp, psz, ppg, pu64, vp, sz, vp]),
+        "sz_encode_reuse_paged_batched": (i32, [i32, i32, vp, ppg, pu64, pvp, psz, vp, vp, sz, vp]),
         "sz_decode": (i32, [i32, vp, sz, vp, u64, vp, sz, vp]),
         "sz_decode_batched": (i32, [i32, i32, pvp, psz, pvp, pu64, vp, sz, vp]),
         "sz_last_device_status": (i32, [vp, vp]),
@@ -242,6 +254,59 @@ def sz_encode_reuse_batched(dtype: int, codebooks: torch.Tensor, xs, outs, ws: t
         "sz_encode_reuse_batched")
 
 
+def paged(dtype: int, pool: torch.Tensor, pages: torch.Tensor, page_elems: int, page_bytes: int = None,
+          pool_pages: int = None) -> sz_paged_t:
+    """Descriptor of a tensor held in pages of `pool` (a contiguous device tensor):
+    `pages` (device int32) lists its page ids in element order, each page holds
+    `page_elems` of its elements, and pages are `page_bytes` apart (default
+    page_elems x element bytes).  The pool, the page table and the descriptor's
+    numbers must stay as they are while a call that uses it runs."""
+    if pages.dtype != torch.int32:
+        raise TypeError("page ids are int32")
+    pb = page_elems * elem_bytes(dtype) if page_bytes is None else int(page_bytes)
+    npages = pool.nbytes // pb if pool_pages is None else int(pool_pages)
+    d = sz_paged_t(_ptr(pool), _ptr(pages), npages, pb, int(page_elems))
+    d._refs = (pool, pages)  # the descriptor keeps the pool and the page table alive
+    return d
+
+
+def _paged_arr(descs):
+    descs = list(descs)
+    return (sz_paged_t * len(descs))(*descs)
+
+
+def sz_plan_paged_batched(dtype: int, srcs, ns, ws: torch.Tensor, plans: torch.Tensor, stream=None):
+    """Plans of T paged tensors (descriptors from paged(); ns: element counts)."""
+    srcs, ns = list(srcs), [int(v) for v in ns]
+    _check(lib.sz_plan_paged_batched(dtype, len(srcs), _paged_arr(srcs), _arr(ctypes.c_uint64, ns), _p(ws),
+                                     ws.nbytes, _p(plans), _stream(stream)), "sz_plan_paged_batched")
+
+
+def sz_encode_paged_batched(dtype: int, plans: torch.Tensor, srcs, ns, outs, ws: torch.Tensor, stream=None):
+    srcs, ns, outs = list(srcs), [int(v) for v in ns], list(outs)
+    _check(lib.sz_encode_paged_batched(dtype, len(srcs), _p(plans), _paged_arr(srcs), _arr(ctypes.c_uint64, ns),
+                                       _arr(ctypes.c_void_p, [_ptr(o) for o in outs]),
+                                       _arr(ctypes.c_size_t, [o.nbytes for o in outs]), _p(ws), ws.nbytes,
+                                       _stream(stream)), "sz_encode_paged_batched")
+
+
+def sz_encode_reuse_paged_batched(dtype: int, codebooks: torch.Tensor, srcs, ns, outs, ws: torch.Tensor,
+                                  totals: torch.Tensor = None, stream=None):
+    srcs, ns, outs = list(srcs), [int(v) for v in ns], list(outs)
+    _check(lib.sz_encode_reuse_paged_batched(
+        dtype, len(srcs), _p(codebooks), _paged_arr(srcs), _arr(ctypes.c_uint64, ns),
+        _arr(ctypes.c_void_p, [_ptr(o) for o in outs]), _arr(ctypes.c_size_t, [o.nbytes for o in outs]),
+        _opt(totals), _p(ws), ws.nbytes, _stream(stream)), "sz_encode_reuse_paged_batched")
+
+
+def sz_decode_paged_batched(dtype: int, comps, dsts, ns, ws: torch.Tensor, comp_bytes=None, stream=None):
+    comps, dsts, ns = list(comps), list(dsts), [int(v) for v in ns]
+    cbs = [c.nbytes for c in comps] if comp_bytes is None else [int(b) for b in comp_bytes]
+    _check(lib.sz_decode_paged_batched(dtype, len(comps), _arr(ctypes.c_void_p, [_ptr(c) for c in comps]),
+                                       _arr(ctypes.c_size_t, cbs), _paged_arr(dsts), _arr(ctypes.c_uint64, ns),
+                                       _p(ws), ws.nbytes, _stream(stream)), "sz_decode_paged_batched")
+
+
 def sz_decode(dtype: int, comp: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, comp_bytes=None,
               stream=None):
     cb = comp.nbytes if comp_bytes is None else int(comp_bytes)
@@ -276,8 +341,28 @@ class Batch:
     """
 
     def __init__(self, dtype: int, xs, outs, ws: torch.Tensor, plans: torch.Tensor, decs=None,
-                 comp_bytes=None):
-        xs, outs = list(xs), list(outs)
+                 comp_bytes=None, src_pages=None, dst_pages=None, n=None):
+        """src_pages / dst_pages: paged() descriptors of the inputs / decode outputs
+        (then xs / decs are not read, and n gives the element counts)."""
+        outs = list(outs)
+        self._src_pages = None if src_pages is None else _paged_arr(src_pages)
+        self._dst_pages = None if dst_pages is None else _paged_arr(dst_pages)
+        if src_pages is not None or dst_pages is not None:
+            if n is None:
+                raise ValueError("paged batches need the element counts n")
+            ns = [int(v) for v in n]
+            self.dtype, self.T = int(dtype), len(outs)
+            self._keep = (xs, outs, decs, ws, plans, src_pages, dst_pages)
+            self._n = self._dn = _arr(ctypes.c_uint64, ns)
+            self._in = None if xs is None else _arr(ctypes.c_void_p, [_ptr(x) for x in xs])
+            self._dec = None if decs is None else _arr(ctypes.c_void_p, [_ptr(d) for d in decs])
+            self._out = _arr(ctypes.c_void_p, [_ptr(o) for o in outs])
+            self._cap = _arr(ctypes.c_size_t, [o.nbytes for o in outs])
+            cbs = [o.nbytes for o in outs] if comp_bytes is None else [int(b) for b in comp_bytes]
+            self._cb = _arr(ctypes.c_size_t, cbs)
+            self._ws, self._wsb, self._plans = _p(ws), ws.nbytes, _p(plans)
+            return
+        xs = list(xs)
         decs = xs if decs is None else list(decs)
         if not (len(xs) == len(outs) == len(decs)) or not 1 <= len(xs) <= SZ_MAX_BATCH:
             raise ValueError("xs, outs and decs must have the same length, 1..%d" % SZ_MAX_BATCH)
@@ -296,10 +381,19 @@ class Batch:
         self._ws, self._wsb, self._plans = _p(ws), ws.nbytes, _p(plans)
 
     def plan(self, stream=None):
+        if self._src_pages is not None:
+            _check(lib.sz_plan_paged_batched(self.dtype, self.T, self._src_pages, self._n, self._ws, self._wsb,
+                                             self._plans, _stream(stream)), "sz_plan_paged_batched")
+            return
         _check(lib.sz_plan_batched(self.dtype, self.T, self._in, self._n, self._ws, self._wsb,
                                    self._plans, _stream(stream)), "sz_plan_batched")
 
     def encode(self, stream=None):
+        if self._src_pages is not None:
+            _check(lib.sz_encode_paged_batched(self.dtype, self.T, self._plans, self._src_pages, self._n,
+                                               self._out, self._cap, self._ws, self._wsb, _stream(stream)),
+                   "sz_encode_paged_batched")
+            return
         _check(lib.sz_encode_batched(self.dtype, self.T, self._plans, self._in, self._n, self._out,
                                      self._cap, self._ws, self._wsb, _stream(stream)), "sz_encode_batched")
 
@@ -309,11 +403,20 @@ class Batch:
         cbs = self._plans if codebooks is None else _p(codebooks)
         if codebooks is not None:
             self._keep_cb = codebooks
+        if self._src_pages is not None:
+            _check(lib.sz_encode_reuse_paged_batched(self.dtype, self.T, cbs, self._src_pages, self._n, self._out,
+                                                     self._cap, _opt(totals), self._ws, self._wsb,
+                                                     _stream(stream)), "sz_encode_reuse_paged_batched")
+            return
         _check(lib.sz_encode_reuse_batched(self.dtype, self.T, cbs, self._in, self._n, self._out, self._cap,
                                            _opt(totals), self._ws, self._wsb, _stream(stream)),
                "sz_encode_reuse_batched")
 
     def decode(self, stream=None):
+        if self._dst_pages is not None:
+            _check(lib.sz_decode_paged_batched(self.dtype, self.T, self._out, self._cb, self._dst_pages, self._dn,
+                                               self._ws, self._wsb, _stream(stream)), "sz_decode_paged_batched")
+            return
         _check(lib.sz_decode_batched(self.dtype, self.T, self._out, self._cb, self._dec, self._dn,
                                      self._ws, self._wsb, _stream(stream)), "sz_decode_batched")
 

@@ -100,6 +100,7 @@ sz_status sz_plan_batched(sz_dtype dtype, int T, const void *const *d_in, const 
     a.hist = reinterpret_cast<uint32_t *>(ws + w.hist);
     a.ticket = reinterpret_cast<uint32_t *>(ws + w.ticket);
     a.plans = reinterpret_cast<uint8_t *>(d_plans);
+    a.paged = nullptr;
     return launch_plan(a, stream);
 }
 
@@ -135,7 +136,7 @@ namespace {
 // codebooks only).
 sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
                         const uint64_t *n, void *const *d_out, const size_t *out_cap, uint64_t *d_totals,
-                        bool reuse, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+                        bool reuse, const sz_paged_t *paged, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
     sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
     if (s != SZ_OK) return s;
     if (!d_plans || !aligned(d_plans, 8) || !d_in || !d_out || !out_cap) return SZ_ERR_INVALID_ARG;
@@ -162,6 +163,7 @@ sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const v
     a.status = reinterpret_cast<unsigned long long *>(ws + w.status);
     a.totals = reinterpret_cast<unsigned long long *>(d_totals);
     a.reuse = reuse ? 1 : 0;
+    a.paged = paged;
     return launch_encode(a, stream);
 }
 
@@ -171,7 +173,8 @@ sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
                             const void *const *d_in, const uint64_t *n, void *const *d_out,
                             const size_t *out_cap, void *d_ws, size_t ws_bytes,
                             cudaStream_t stream) {
-    return encode_common(dtype, T, d_plans, d_in, n, d_out, out_cap, nullptr, false, d_ws, ws_bytes, stream);
+    return encode_common(dtype, T, d_plans, d_in, n, d_out, out_cap, nullptr, false, nullptr, d_ws, ws_bytes,
+                         stream);
 }
 
 sz_status sz_encode(sz_dtype dtype, const sz_plan_t *d_plan, const void *d_in, uint64_t n,
@@ -185,8 +188,8 @@ sz_status sz_encode_reuse_batched(sz_dtype dtype, int T, const sz_plan_t *d_code
                                   const void *const *d_in, const uint64_t *n, void *const *d_out,
                                   const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
                                   cudaStream_t stream) {
-    return encode_common(dtype, T, d_codebooks, d_in, n, d_out, out_cap, d_totals, true, d_ws, ws_bytes,
-                         stream);
+    return encode_common(dtype, T, d_codebooks, d_in, n, d_out, out_cap, d_totals, true, nullptr, d_ws,
+                         ws_bytes, stream);
 }
 
 sz_status sz_encode_reuse(sz_dtype dtype, const sz_plan_t *d_codebook, const void *d_in, uint64_t n,
@@ -198,9 +201,11 @@ sz_status sz_encode_reuse(sz_dtype dtype, const sz_plan_t *d_codebook, const voi
                                    stream);
 }
 
-sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,
-                            const size_t *comp_bytes, void *const *d_out, const uint64_t *n,
-                            void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+namespace {
+
+sz_status decode_common(sz_dtype dtype, int T, const void *const *d_comp, const size_t *comp_bytes,
+                        void *const *d_out, const uint64_t *n, const sz_paged_t *paged, void *d_ws,
+                        size_t ws_bytes, cudaStream_t stream) {
     sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
     if (s != SZ_OK) return s;
     if (!d_comp || !comp_bytes || !d_out) return SZ_ERR_INVALID_ARG;
@@ -219,7 +224,16 @@ sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,
     a.out = d_out;
     a.n = n;
     a.ctl = static_cast<uint32_t *>(d_ws);
+    a.paged = paged;
     return launch_decode(a, stream);
+}
+
+}  // namespace
+
+sz_status sz_decode_batched(sz_dtype dtype, int T, const void *const *d_comp,
+                            const size_t *comp_bytes, void *const *d_out, const uint64_t *n,
+                            void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    return decode_common(dtype, T, d_comp, comp_bytes, d_out, n, nullptr, d_ws, ws_bytes, stream);
 }
 
 sz_status sz_decode(sz_dtype dtype, const void *d_comp, size_t comp_bytes, void *d_out, uint64_t n,
@@ -242,3 +256,99 @@ sz_status sz_last_device_status(void *d_ws, cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------- paged tensors
+
+namespace sz {
+
+PageRef page_ref(const sz_paged_t *d) {
+    PageRef r;
+    r.pages = d ? d->pages : nullptr;
+    r.pool_pages = d ? d->pool_pages : 0;
+    r.page_bytes = d ? d->page_bytes : 0;
+    r.page_elems = d ? d->page_elems : 0;
+    return r;
+}
+
+}  // namespace sz
+
+namespace {
+
+// Host checks of T page descriptors; fills pools[t] with each pool's base.
+sz_status check_paged(sz_dtype dtype, int T, const sz_paged_t *pg, const uint64_t *n, const void **pools) {
+    if (!pg || !n || T < 1 || T > SZ_MAX_BATCH) return SZ_ERR_INVALID_ARG;
+    const uint64_t eb = dtype == SZ_BF16 ? 2 : 1;
+    for (int t = 0; t < T; ++t) {
+        const sz_paged_t &d = pg[t];
+        pools[t] = d.pool;
+        if (n[t] == 0) continue;
+        if (!d.pool || !aligned(d.pool, 16) || !d.pages || !aligned(d.pages, 4) || d.pool_pages == 0)
+            return SZ_ERR_INVALID_ARG;
+        if (d.page_elems == 0 || d.page_elems % 1024u != 0 || d.page_bytes % 16 != 0 ||
+            d.page_bytes < uint64_t(d.page_elems) * eb)
+            return SZ_ERR_INVALID_ARG;
+    }
+    return SZ_OK;
+}
+
+}  // namespace
+
+sz_status sz_plan_paged_batched(sz_dtype dtype, int T, const sz_paged_t *src, const uint64_t *n,
+                                void *d_ws, size_t ws_bytes, sz_plan_t *d_plans, cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return SZ_ERR_UNSUPPORTED_DTYPE;
+    const void *pools[SZ_MAX_BATCH];
+    sz_status s = check_paged(dtype, T, src, n, pools);
+    if (s != SZ_OK) return s;
+    s = check_batch(dtype, T, n, d_ws, ws_bytes);
+    if (s != SZ_OK) return s;
+    if (!d_plans || !aligned(d_plans, 8)) return SZ_ERR_INVALID_ARG;
+    const WsLayout w = ws_layout(T, total_tiles(T, n));
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    PlanArgs a;
+    a.dtype = dtype;
+    a.T = T;
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return SZ_ERR_CUDA;
+    a.in = pools;
+    a.n = n;
+    a.ctl = reinterpret_cast<uint32_t *>(ws);
+    a.hist = reinterpret_cast<uint32_t *>(ws + w.hist);
+    a.ticket = reinterpret_cast<uint32_t *>(ws + w.ticket);
+    a.plans = reinterpret_cast<uint8_t *>(d_plans);
+    a.paged = src;
+    return launch_plan(a, stream);
+}
+
+sz_status sz_encode_paged_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans, const sz_paged_t *src,
+                                  const uint64_t *n, void *const *d_out, const size_t *out_cap, void *d_ws,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return SZ_ERR_UNSUPPORTED_DTYPE;
+    const void *pools[SZ_MAX_BATCH];
+    sz_status s = check_paged(dtype, T, src, n, pools);
+    if (s != SZ_OK) return s;
+    return encode_common(dtype, T, d_plans, pools, n, d_out, out_cap, nullptr, false, src, d_ws, ws_bytes, stream);
+}
+
+sz_status sz_decode_paged_batched(sz_dtype dtype, int T, const void *const *d_comp, const size_t *comp_bytes,
+                                  const sz_paged_t *dst, const uint64_t *n, void *d_ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return SZ_ERR_UNSUPPORTED_DTYPE;
+    const void *pools[SZ_MAX_BATCH];
+    sz_status s = check_paged(dtype, T, dst, n, pools);
+    if (s != SZ_OK) return s;
+    void *outs[SZ_MAX_BATCH];
+    for (int t = 0; t < T; ++t) outs[t] = const_cast<void *>(pools[t]);
+    return decode_common(dtype, T, d_comp, comp_bytes, outs, n, dst, d_ws, ws_bytes, stream);
+}
+
+sz_status sz_encode_reuse_paged_batched(sz_dtype dtype, int T, const sz_plan_t *d_codebooks,
+                                        const sz_paged_t *src, const uint64_t *n, void *const *d_out,
+                                        const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
+                                        cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return SZ_ERR_UNSUPPORTED_DTYPE;
+    const void *pools[SZ_MAX_BATCH];
+    sz_status s = check_paged(dtype, T, src, n, pools);
+    if (s != SZ_OK) return s;
+    return encode_common(dtype, T, d_codebooks, pools, n, d_out, out_cap, d_totals, true, src, d_ws, ws_bytes,
+                         stream);
+}

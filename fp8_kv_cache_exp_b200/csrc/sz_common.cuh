@@ -133,6 +133,16 @@ inline WsLayout ws_layout(int T, uint64_t total_tiles) {
 // ------------------------------------------------------------- parameters
 // Passed by value as __grid_constant__ kernel parameters: no descriptor copy.
 
+// Where a tensor's elements live: contiguous at its base pointer (pages ==
+// nullptr), or in pages of a pool at that base -- element i at
+// base + pages[i / page_elems] * page_bytes + (i % page_elems) * element bytes.
+struct PageRef {
+    const int32_t *pages;
+    uint64_t pool_pages;
+    uint64_t page_bytes;
+    uint32_t page_elems;  // a multiple of 1024 (a quarter block never straddles pages)
+};
+
 template <int MAXB>
 struct PlanParams {
     uint32_t *ctl;
@@ -144,6 +154,7 @@ struct PlanParams {
     const uint8_t *in[MAXB];
     uint64_t n[MAXB];
     uint64_t item_begin[MAXB + 1];  // prefix over tensors of ceil(n / item elements)
+    PageRef pg[MAXB];
 };
 
 // Encode and decode work in chunks: up to kMaxChunkBlocks consecutive
@@ -169,6 +180,7 @@ struct EncodeParams {
     uint64_t cap[MAXB];
     uint32_t chunk_begin[MAXB + 1];  // prefix over tensors of their chunk counts
     uint16_t empty[MAXB];
+    PageRef pg[MAXB];                // input pages
 };
 
 template <int MAXB>
@@ -182,6 +194,7 @@ struct DecodeParams {
     uint8_t *out[MAXB];
     uint64_t n[MAXB];
     uint32_t block_begin[MAXB + 1];  // prefix over tensors of their 4096-element blocks
+    PageRef pg[MAXB];                // output pages
 };
 
 // Blocks per chunk for a launch: the largest power of two (<= kMaxChunkBlocks)
@@ -197,6 +210,19 @@ inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_ctas) {
 // Record the first device error; later errors keep the first one.
 __device__ inline void set_error(uint32_t *ctl, uint32_t code, uint32_t detail) {
     if (atomicCAS(&ctl[kCtlErr], 0u, code) == 0u) atomicExch(&ctl[kCtlErrDetail], detail);
+}
+
+// Byte offset of element e from its tensor's base (PageRef above), or
+// kBadOffset when the page id is outside the pool.  For paged tensors this
+// reads one page id (read-only path).
+constexpr uint64_t kBadOffset = ~0ull;
+template <int EB>
+__device__ __forceinline__ uint64_t elem_offset(const PageRef &pr, uint64_t e) {
+    if (!pr.pages) return e * EB;
+    const uint32_t page = uint32_t(e) / pr.page_elems;  // e < 2^32: tensors hold fewer than 2^32 elements
+    const int64_t id = __ldg(pr.pages + page);
+    if (id < 0 || uint64_t(id) >= pr.pool_pages) return kBadOffset;
+    return uint64_t(id) * pr.page_bytes + (e - uint64_t(page) * pr.page_elems) * EB;
 }
 
 __device__ inline uint64_t global_ns() {

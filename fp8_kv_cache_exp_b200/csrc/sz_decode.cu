@@ -239,10 +239,10 @@ __device__ __forceinline__ void patch(uint32_t (&o)[4], uint32_t j, uint32_t e) 
 // Decode one step.  running: escapes of the block before this step (updated);
 // esc_reg: lane i holds the block's escape i (i < 32); esc_g: the block's
 // escapes in global memory; cnt: escapes the offsets table gives the block.
-template <int DT, bool PARTIAL>
+template <int DT, bool PARTIAL, bool CHECKED = false>
 __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const uint32_t (&xt)[4],
                                             uint8_t *dst, int valid, uint32_t &running, uint32_t esc_reg,
-                                            const uint8_t *esc_g, uint32_t cnt, bool &bad) {
+                                            const uint8_t *esc_g, uint32_t cnt, bool &bad, bool store = true) {
     uint32_t o[4];
     // escape flags of this lane's elements: bit 4j for element j
     typename std::conditional<DT == SZ_BF16, uint32_t, uint64_t>::type m;
@@ -317,7 +317,9 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
         }
         running += tot;
     }
-    if (!PARTIAL) {
+    if (CHECKED && !store) {
+        // an output page outside the pool: nothing is written
+    } else if (!PARTIAL) {
         *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
     } else if constexpr (DT == SZ_BF16) {
 #pragma unroll
@@ -447,8 +449,8 @@ struct QuarterFeed {
     }
 };
 
-template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
+template <int DT, int MAXB, bool PAGED>
+__device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
     using G = DGeo<DT>;
     extern __shared__ __align__(128) uint8_t s_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -496,8 +498,15 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
             const bool ok = ws.ok && offsets_ok(be, ws, blk);
             const uint32_t cnt = ok ? be.hi - be.lo : 0u;
             const uint8_t *esc_g = comp + ws.esc + be.lo;
-            uint8_t *out = p.out[t] + (uint64_t(blk) * kBlock + uint64_t(lane) * G::LE) * Dt<DT>::kElemBytes;
+            constexpr int EB = Dt<DT>::kElemBytes;
+            uint8_t *out = p.out[t] + (uint64_t(blk) * kBlock + uint64_t(lane) * G::LE) * EB;
             const bool full = (uint64_t(blk) + 1) * kBlock <= ws.n;
+            // paged output: lane q < 4 looks up where quarter q of the block goes
+            uint64_t qoff = 0;
+            if constexpr (PAGED) {
+                if (lane < 4 && uint64_t(blk) * kBlock + uint64_t(lane) * (kBlock / 4) < ws.n)
+                    qoff = elem_offset<EB>(p.pg[t], uint64_t(blk) * kBlock + uint64_t(lane) * (kBlock / 4));
+            }
             uint32_t running = 0;
             bool bad = false, timed_out = false;
             for (int q = 0; q < 4; ++q, ++v) {
@@ -517,11 +526,24 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
                 if (ok && !timed_out) {
                     if (full) {
                         const uint32_t st_addr = smem_u32(W.stage[st]);
+                        if constexpr (PAGED) {
+                            const uint64_t off = __shfl_sync(0xffffffffu, qoff, q);
+                            const bool store = off != kBadOffset;
+                            uint8_t *out_q = p.out[t] + off + uint64_t(lane) * G::LE * EB;
+                            if (!store && lane == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
 #pragma unroll
-                        for (int it = 0; it < G::QIT; ++it) {
-                            const DFrag f = read_stage<DT>(st_addr, it);
-                            decode_step<DT, false>(f, tab_addr, ws.xt, out + (q * G::QIT + it) * 512, G::LE, running,
-                                                   esc_reg, esc_g, cnt, bad);
+                            for (int it = 0; it < G::QIT; ++it) {
+                                const DFrag f = read_stage<DT>(st_addr, it);
+                                decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE, running,
+                                                             esc_reg, esc_g, cnt, bad, store);
+                            }
+                        } else {
+#pragma unroll
+                            for (int it = 0; it < G::QIT; ++it) {
+                                const DFrag f = read_stage<DT>(st_addr, it);
+                                decode_step<DT, false>(f, tab_addr, ws.xt, out + (q * G::QIT + it) * 512, G::LE,
+                                                       running, esc_reg, esc_g, cnt, bad);
+                            }
                         }
                     } else {
                         for (int it = q * G::QIT; it < (q + 1) * G::QIT; ++it) {
@@ -529,8 +551,21 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
                             const int64_t left = int64_t(ws.n) - e;
                             const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
                             const DFrag f = read_partial<DT>(comp, ws, blk, it, valid);
-                            decode_step<DT, true>(f, tab_addr, ws.xt, out + it * 512, valid, running, esc_reg, esc_g, cnt,
-                                                  bad);
+                            if constexpr (PAGED) {
+                                uint8_t *dst = out;
+                                bool store = valid > 0;
+                                if (valid > 0) {
+                                    const uint64_t off = elem_offset<EB>(p.pg[t], uint64_t(e));
+                                    store = off != kBadOffset;
+                                    dst = p.out[t] + off;
+                                    if (!store) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
+                                }
+                                decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg, esc_g,
+                                                            cnt, bad, store);
+                            } else {
+                                decode_step<DT, true>(f, tab_addr, ws.xt, out + it * 512, valid, running, esc_reg,
+                                                      esc_g, cnt, bad);
+                            }
                         }
                     }
                 }
@@ -572,9 +607,21 @@ __global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ Deco
     }
 }
 
+// Contiguous outputs: ptxas keeps this kernel at 80 registers on its own.
 template <int DT, int MAXB>
+__global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
+    decode_body<DT, MAXB, false>(p);
+}
+
+// Paged outputs: capped for three CTAs per SM.
+template <int DT, int MAXB>
+__global__ void __launch_bounds__(NT, 3) decode_kernel_paged(const __grid_constant__ DecodeParams<MAXB> p) {
+    decode_body<DT, MAXB, true>(p);
+}
+
+template <int DT, int MAXB, bool PAGED>
 sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
-    auto kern = decode_kernel<DT, MAXB>;
+    auto kern = PAGED ? decode_kernel_paged<DT, MAXB> : decode_kernel<DT, MAXB>;
     const size_t smem = sizeof(WarpSmem) * NW;
     static std::atomic<int> cache[kMaxDevices];
     const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
@@ -582,6 +629,7 @@ sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     DecodeParams<MAXB> p;
     p.ctl = a.ctl;
     p.claim = a.ctl + kCtlWords;  // the histogram slots
+    for (int t = 0; t < a.T; ++t) p.pg[t] = page_ref(a.paged ? a.paged + t : nullptr);
     p.T = a.T;
     p.block_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
@@ -604,11 +652,19 @@ sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 sz_status launch_decode(const DecodeArgs &a, cudaStream_t stream) {
+    // paged outputs get their own instantiation: contiguous ones carry no paging code
+    if (a.paged) {
+        if (a.dtype == SZ_BF16)
+            return a.T <= kSmallBatch ? launch_decode_t<SZ_BF16, kSmallBatch, true>(a, stream)
+                                      : launch_decode_t<SZ_BF16, kLargeBatch, true>(a, stream);
+        return a.T <= kSmallBatch ? launch_decode_t<SZ_FP8_E5M2, kSmallBatch, true>(a, stream)
+                                  : launch_decode_t<SZ_FP8_E5M2, kLargeBatch, true>(a, stream);
+    }
     if (a.dtype == SZ_BF16)
-        return a.T <= kSmallBatch ? launch_decode_t<SZ_BF16, kSmallBatch>(a, stream)
-                                  : launch_decode_t<SZ_BF16, kLargeBatch>(a, stream);
-    return a.T <= kSmallBatch ? launch_decode_t<SZ_FP8_E5M2, kSmallBatch>(a, stream)
-                              : launch_decode_t<SZ_FP8_E5M2, kLargeBatch>(a, stream);
+        return a.T <= kSmallBatch ? launch_decode_t<SZ_BF16, kSmallBatch, false>(a, stream)
+                                  : launch_decode_t<SZ_BF16, kLargeBatch, false>(a, stream);
+    return a.T <= kSmallBatch ? launch_decode_t<SZ_FP8_E5M2, kSmallBatch, false>(a, stream)
+                              : launch_decode_t<SZ_FP8_E5M2, kLargeBatch, false>(a, stream);
 }
 
 }  // namespace sz

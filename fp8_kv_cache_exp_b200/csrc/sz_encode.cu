@@ -416,8 +416,8 @@ __device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &runnin
 // One warp codes block blk of a tensor of n elements: planes and codes go to
 // out; escapes (exponents in element order) go to put(rank, exponent).
 // Returns the block's escape count.
-template <int DT, bool STORE, typename Put>
-__device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, uint64_t n,
+template <int DT, bool STORE, bool PAGED, typename Put>
+__device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, const PageRef &pr, uint64_t n,
                                                uint64_t blk, const Layout &L, uint8_t *out, Put put) {
     using G = Geo<DT>;
     const int lane = threadIdx.x & 31;
@@ -425,7 +425,20 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
     const EPtr q = block_out<DT>(out, L, e_lane);
     uint32_t running = 0;
-    if ((blk + 1) * kBlock <= n) {
+    if (PAGED && pr.pages) {
+        // paged input: each step's 16 bytes from its own page (a step never straddles one)
+        for (int it = 0; it < G::IT; ++it) {
+            const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
+            const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (valid > 0) {
+                const uint64_t off = elem_offset<Dt<DT>::kElemBytes>(pr, e_lane + uint64_t(it) * 32 * G::LE);
+                if (off != kBadOffset) v = load_step<DT>(in + off, valid);
+            }
+            const EMask<DT> m = code_step<DT, STORE>(lut, v, valid, q, it);
+            rank_step<DT>(m, v, running, put);
+        }
+    } else if ((blk + 1) * kBlock <= n) {
         uint4 ring[G::kAhead + 1];
 #pragma unroll
         for (int i = 0; i < G::kAhead; ++i) ring[i] = __ldcs(reinterpret_cast<const uint4 *>(src + i * 512));
@@ -461,18 +474,23 @@ struct RingState {
 
 template <int DT>
 __device__ __forceinline__ void ring_issue(WarpShared &W, RingState &R, const uint8_t *in, uint64_t n,
-                                           uint64_t b0, uint32_t x) {
+                                           uint64_t b0, uint32_t x, bool paged, uint64_t paged_off, uint32_t *ctl) {
     constexpr uint32_t kQB = kBlock / 4 * Dt<DT>::kElemBytes;  // bytes of a quarter block
     const int st = int(R.vi % kRing);
     const uint64_t blk = b0 + x / 4;
     if ((blk + 1) * kBlock <= n) {
-        if ((threadIdx.x & 31) == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&W.bar[st], kQB);
-            bulk_g2s(W.ring[st], in + (blk * kBlock + (x % 4) * (kBlock / 4)) * Dt<DT>::kElemBytes, kQB,
-                     &W.bar[st]);
+        // byte offset of the quarter from the input base (paged: looked up by the caller)
+        const uint64_t off = paged ? paged_off : (blk * kBlock + (x % 4) * (kBlock / 4)) * Dt<DT>::kElemBytes;
+        if (off != kBadOffset) {
+            if ((threadIdx.x & 31) == 0) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&W.bar[st], kQB);
+                bulk_g2s(W.ring[st], in + off, kQB, &W.bar[st]);
+            }
+            R.issued |= 1u << st;
+        } else if ((threadIdx.x & 31) == 0) {
+            set_error(ctl, SZ_ERR_INVALID_ARG, uint32_t(blk));  // page id outside the pool: not read
         }
-        R.issued |= 1u << st;
     }
     ++R.vi;
 }
@@ -535,7 +553,7 @@ __device__ __forceinline__ ChunkGeo chunk_geo(const EncodeParams<MAXB> &p, uint3
 // esc[slot] (element order) with per-block offsets in blk_off[slot].  Between
 // blocks it calls between().  Returns the chunk's escape count, or
 // 0xFFFFFFFF if the plan does not fit the data (reported; nothing to finish).
-template <int DT, int MAXB, typename Between>
+template <int DT, int MAXB, bool PAGED, typename Between>
 __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
                                WarpShared &W, RingState &R, int &plan_tensor, bool *lost, Between between) {
     const int lane = threadIdx.x & 31;
@@ -559,8 +577,18 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
     constexpr int QIT = G::IT / 4;  // steps per quarter block
     const uint32_t lut = lut_addr(W), stage = smem_u32(W.esc[slot]);
     const uint32_t nunits = 4u * uint32_t(nbk);
+    // paged input: lane x looks up where unit x (a quarter block) of the chunk lives
+    const PageRef &pr = p.pg[g.t];
+    const bool paged = PAGED && pr.pages != nullptr;
+    uint64_t unit_off = 0;
+    if (paged && uint32_t(lane) < nunits && b0 * kBlock + uint64_t(lane) * (kBlock / 4) < n)
+        unit_off = elem_offset<Dt<DT>::kElemBytes>(pr, b0 * kBlock + uint64_t(lane) * (kBlock / 4));
+    auto issue = [&](uint32_t x) {
+        const uint64_t off = paged ? __shfl_sync(0xffffffffu, unit_off, int(x)) : 0ull;
+        ring_issue<DT>(W, R, in, n, b0, x, paged, off, p.ctl);
+    };
     uint32_t next_x = 0;
-    for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) ring_issue<DT>(W, R, in, n, b0, next_x);
+    for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) issue(next_x);
     uint32_t running = 0;
 #pragma unroll 1
     for (int k = 0; k < nbk; ++k) {
@@ -576,7 +604,7 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
         uint32_t blk_run = 0;
 #pragma unroll 1
         for (int qq = 0; qq < 4; ++qq) {
-            if (next_x < nunits) ring_issue<DT>(W, R, in, n, b0, next_x++);
+            if (next_x < nunits) issue(next_x++);
             int st;
             *lost = !ring_take(W, R, &st) || *lost;
             if (full) {
@@ -588,11 +616,15 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
                     rank_step<DT>(m, v, blk_run, put);
                 }
             } else {
-                const uint8_t *src = in + e_lane * Dt<DT>::kElemBytes;
                 for (int it = qq * QIT; it < (qq + 1) * QIT; ++it) {
                     const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
                     const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
-                    const uint4 v = valid > 0 ? load_step<DT>(src + it * 512, valid) : make_uint4(0, 0, 0, 0);
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (valid > 0) {
+                        const uint64_t e = e_lane + uint64_t(it) * 32 * G::LE;
+                        const uint64_t off = paged ? elem_offset<Dt<DT>::kElemBytes>(pr, e) : e * Dt<DT>::kElemBytes;
+                        if (off != kBadOffset) v = load_step<DT>(in + off, valid);
+                    }
                     const EMask<DT> m = code_step<DT, true>(lut, v, valid, q, it);
                     rank_step<DT>(m, v, blk_run, put);
                 }
@@ -610,7 +642,7 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
 // escapes (from the stage, or re-coded from the input when they overflowed
 // it -- the warp's code table is then still the chunk's), and the stream
 // frame if it is the tensor's last chunk.
-template <int DT, int MAXB>
+template <int DT, int MAXB, bool PAGED>
 __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
                              uint32_t total, const Lookback &lb, WarpShared &W) {
     const int lane = threadIdx.x & 31;
@@ -639,7 +671,7 @@ __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const Ch
 #pragma unroll 1
         for (int k = 0; k < g.nbk; ++k) {
             const uint64_t d = dst + W.blk_off[slot][k];
-            code_block<DT, false>(lut, p.in[g.t], g.n, g.b0 + k, L, out, [&](uint32_t r, uint32_t e) {
+            code_block<DT, false, PAGED>(lut, p.in[g.t], p.pg[g.t], g.n, g.b0 + k, L, out, [&](uint32_t r, uint32_t e) {
                 if (d + r < bound) out[d + r] = uint8_t(e);
             });
         }
@@ -685,7 +717,7 @@ __device__ __forceinline__ unsigned long long *chunk_status(const EncodeParams<M
     return p.status + p.chunk_begin[t];
 }
 
-template <int DT, int MAXB>
+template <int DT, int MAXB, bool PAGED>
 __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     extern __shared__ __align__(128) uint8_t s_raw[];
     WarpShared *s_warp = reinterpret_cast<WarpShared *>(s_raw);
@@ -710,7 +742,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
         if (!pend.valid) return;
         const ChunkGeo pg = chunk_geo<MAXB>(p, pend.job);
         if (lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, block)) {
-            finish_chunk<DT, MAXB>(p, pend.job, pg, pend.slot, pend.total, pend.lb, W);
+            finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, pend.lb, W);
             pend.valid = false;
         }
     };
@@ -727,7 +759,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
         const ChunkGeo g = chunk_geo<MAXB>(p, job);
         const int slot = pend.valid ? (pend.slot ^ 1) : 0;
         bool lost = false;
-        const uint32_t total = code_chunk<DT, MAXB>(p, job, g, slot, W, R, plan_tensor, &lost,
+        const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost,
                                                     [&]() { settle(false); });
         if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
         if (total == 0xFFFFFFFFu) continue;  // plan rejected for this tensor
@@ -737,7 +769,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
         settle(true);  // at most one chunk waits for its offset
         if (total > kWarpStage || lookback_advance(lb, st, g.chunk, total, tag, false)) {
             lookback_advance(lb, st, g.chunk, total, tag, true);
-            finish_chunk<DT, MAXB>(p, job, g, slot, total, lb, W);
+            finish_chunk<DT, MAXB, PAGED>(p, job, g, slot, total, lb, W);
         } else {
             pend.valid = true;
             pend.job = job;
@@ -759,9 +791,9 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
     }
 }
 
-template <int DT, int MAXB>
+template <int DT, int MAXB, bool PAGED>
 sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
-    auto kern = encode_kernel<DT, MAXB>;
+    auto kern = encode_kernel<DT, MAXB, PAGED>;
     const size_t smem = sizeof(WarpShared) * NW;
     static std::atomic<int> cache[kMaxDevices];
     const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
@@ -773,6 +805,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     p.plans = a.plans;
     p.totals = a.totals;
     p.reuse = a.reuse;
+    for (int t = 0; t < a.T; ++t) p.pg[t] = page_ref(a.paged ? a.paged + t : nullptr);
     p.T = a.T;
     p.n_empty = 0;
     p.chunk_log2 = 3;  // kChunkBlocks
@@ -798,11 +831,19 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 sz_status launch_encode(const EncodeArgs &a, cudaStream_t stream) {
+    // paged inputs get their own instantiation: contiguous ones carry no paging code
+    if (a.paged) {
+        if (a.dtype == SZ_BF16)
+            return a.T <= kSmallBatch ? launch_encode_t<SZ_BF16, kSmallBatch, true>(a, stream)
+                                      : launch_encode_t<SZ_BF16, kLargeBatch, true>(a, stream);
+        return a.T <= kSmallBatch ? launch_encode_t<SZ_FP8_E5M2, kSmallBatch, true>(a, stream)
+                                  : launch_encode_t<SZ_FP8_E5M2, kLargeBatch, true>(a, stream);
+    }
     if (a.dtype == SZ_BF16)
-        return a.T <= kSmallBatch ? launch_encode_t<SZ_BF16, kSmallBatch>(a, stream)
-                                  : launch_encode_t<SZ_BF16, kLargeBatch>(a, stream);
-    return a.T <= kSmallBatch ? launch_encode_t<SZ_FP8_E5M2, kSmallBatch>(a, stream)
-                              : launch_encode_t<SZ_FP8_E5M2, kLargeBatch>(a, stream);
+        return a.T <= kSmallBatch ? launch_encode_t<SZ_BF16, kSmallBatch, false>(a, stream)
+                                  : launch_encode_t<SZ_BF16, kLargeBatch, false>(a, stream);
+    return a.T <= kSmallBatch ? launch_encode_t<SZ_FP8_E5M2, kSmallBatch, false>(a, stream)
+                              : launch_encode_t<SZ_FP8_E5M2, kLargeBatch, false>(a, stream);
 }
 
 }  // namespace sz

@@ -15,6 +15,7 @@ struct PlanArgs {
     const uint64_t *n;
     uint32_t *ctl, *hist, *ticket;
     uint8_t *plans;
+    const sz_paged_t *paged;  // T input page descriptors, or null (contiguous inputs)
 };
 
 struct EncodeArgs {
@@ -28,6 +29,7 @@ struct EncodeArgs {
     unsigned long long *status;
     unsigned long long *totals;  // may be null
     int reuse;                   // codebook reuse: plans give codebooks only
+    const sz_paged_t *paged;     // T input page descriptors, or null (contiguous inputs)
 };
 
 struct DecodeArgs {
@@ -37,7 +39,11 @@ struct DecodeArgs {
     void *const *out;
     const uint64_t *n;
     uint32_t *ctl;
+    const sz_paged_t *paged;  // T output page descriptors, or null (contiguous outputs)
 };
+
+// Kernel page reference of descriptor d (or a contiguous tensor when d is null).
+PageRef page_ref(const sz_paged_t *d);
 
 sz_status launch_plan(const PlanArgs &a, cudaStream_t stream);
 sz_status launch_encode(const EncodeArgs &a, cudaStream_t stream);

@@ -230,8 +230,24 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
         uint32_t *g_hist = p.hist + size_t(t) * 256;
         // sub-ranges short enough that no 16-bit counter can overflow
         constexpr uint64_t kSub = uint64_t(kMaxPerThread / C::kVecElems) * C::kVecElems * NT;
+        const PageRef &pr = p.pg[t];
         for (uint64_t s = a; s < b; s += kSub) {
-            count_range<DT, NT>(col, inc, p.in[t], s, min(b, s + kSub));
+            const uint64_t e = min(b, s + kSub);
+            if (!pr.pages) {
+                count_range<DT, NT>(col, inc, p.in[t], s, e);
+            } else {
+                // a paged tensor: count each page's piece from its own address
+                for (uint64_t x = s; x < e;) {
+                    const uint64_t y = min(e, (x / pr.page_elems + 1) * pr.page_elems);
+                    const uint64_t off = elem_offset<C::kElemBytes>(pr, x);
+                    if (off == kBadOffset) {
+                        if (tid == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, uint32_t(t));
+                    } else {
+                        count_range<DT, NT>(col, inc, p.in[t] + off, 0, y - x);
+                    }
+                    x = y;
+                }
+            }
             flush_columns<DT, NT>(s_cols, g_hist);
         }
         // ticket: the CTA that completes the tensor's last item selects its codebook
@@ -263,6 +279,7 @@ sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
     p.plans = a.plans;
     p.T = a.T;
     p.item_begin[0] = 0;
+    for (int t = 0; t < a.T; ++t) p.pg[t] = page_ref(a.paged ? a.paged + t : nullptr);
     for (int t = 0; t < a.T; ++t) {
         p.in[t] = static_cast<const uint8_t *>(a.in[t]);
         p.n[t] = a.n[t];

@@ -93,6 +93,28 @@ typedef struct {
     unsigned char bytes[SZ_HEADER_BYTES];
 } sz_plan_t;
 
+/* A tensor held in pages of a page pool, as paged KV caches keep it: element
+ * i lives at
+ *     pool + pages[i / page_elems] * page_bytes + (i % page_elems) * elem_bytes
+ * (elem_bytes = 2 for BF16, 1 for E5M2).  All fields are device-side data
+ * described by the host; the descriptor itself is read on the host during the
+ * call.
+ *   pool        device base of the pool, 16-byte aligned
+ *   pages       device array of ceil(n / page_elems) page ids, in element order
+ *   pool_pages  number of pages in the pool; an id outside [0, pool_pages) is
+ *               reported as SZ_ERR_INVALID_ARG on the device error word and
+ *               that page is neither read nor written
+ *   page_bytes  bytes from one page to the next, a multiple of 16 and at least
+ *               page_elems * elem_bytes
+ *   page_elems  elements of this tensor per page, a multiple of 1024 */
+typedef struct {
+    const void *pool;
+    const int32_t *pages;
+    uint64_t pool_pages;
+    uint64_t page_bytes;
+    uint32_t page_elems;
+} sz_paged_t;
+
 /* ------------------------------------------------------------ host-only */
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -185,6 +207,27 @@ sz_status sz_encode_reuse_batched(sz_dtype dtype, int T, const sz_plan_t *d_code
                                   const void *const *d_in, const uint64_t *n, void *const *d_out,
                                   const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
                                   cudaStream_t stream);
+
+/* Paged tensors (see sz_paged_t): the same three steps for tensors held in
+ * the pages of a page pool -- the stream of a paged tensor is the stream of
+ * its elements taken in order, as if gathered into one contiguous tensor.
+ * src / dst are HOST arrays of T descriptors; everything else is as in the
+ * contiguous calls.  Decode writes only the bytes of the tensor's elements
+ * inside its pages. */
+sz_status sz_plan_paged_batched(sz_dtype dtype, int T, const sz_paged_t *src, const uint64_t *n,
+                                void *d_ws, size_t ws_bytes, sz_plan_t *d_plans, cudaStream_t stream);
+sz_status sz_encode_paged_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans, const sz_paged_t *src,
+                                  const uint64_t *n, void *const *d_out, const size_t *out_cap, void *d_ws,
+                                  size_t ws_bytes, cudaStream_t stream);
+sz_status sz_decode_paged_batched(sz_dtype dtype, int T, const void *const *d_comp, const size_t *comp_bytes,
+                                  const sz_paged_t *dst, const uint64_t *n, void *d_ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+/* Codebook reuse (sz_encode_reuse_batched) for paged inputs. */
+sz_status sz_encode_reuse_paged_batched(sz_dtype dtype, int T, const sz_plan_t *d_codebooks,
+                                        const sz_paged_t *src, const uint64_t *n, void *const *d_out,
+                                        const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
+                                        cudaStream_t stream);
 
 /* Decode a stream of comp_bytes bytes holding n elements of dtype into d_out
  * (BF16: 2n bytes, E5M2: n bytes); the result is bitwise identical to the
