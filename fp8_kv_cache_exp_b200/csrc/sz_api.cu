@@ -284,7 +284,7 @@ sz_status check_paged(sz_dtype dtype, int T, const sz_paged_t *pg, const uint64_
         if (n[t] == 0) continue;
         if (!d.pool || !aligned(d.pool, 16) || !d.pages || !aligned(d.pages, 4) || d.pool_pages == 0)
             return SZ_ERR_INVALID_ARG;
-        if (d.page_elems == 0 || d.page_elems % 1024u != 0 || d.page_bytes % 16 != 0 ||
+        if (d.page_elems == 0 || d.page_elems % 1024u != 0 || d.page_elems > (1u << 18) || d.page_bytes % 16 != 0 ||
             d.page_bytes < uint64_t(d.page_elems) * eb)
             return SZ_ERR_INVALID_ARG;
     }

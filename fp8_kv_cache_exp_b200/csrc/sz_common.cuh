@@ -140,7 +140,7 @@ struct PageRef {
     const int32_t *pages;
     uint64_t pool_pages;
     uint64_t page_bytes;
-    uint32_t page_elems;  // a multiple of 1024 (a quarter block never straddles pages)
+    uint32_t page_elems;  // a multiple of 1024 (a quarter block never straddles pages), <= 2^18
 };
 
 template <int MAXB>

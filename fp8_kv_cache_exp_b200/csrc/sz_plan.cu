@@ -105,6 +105,79 @@ __device__ void count_range(uint32_t *col, uint32_t inc, const uint8_t *in, uint
     }
 }
 
+// Page ids cached in shared memory per pass of count_range_paged.
+constexpr uint32_t kPageCache = 4096;
+
+// Count elements [a, b) of a paged tensor (a a multiple of the vector size);
+// called by the whole CTA.  The range's page ids are first copied into shared
+// memory (s_ids, kPageCache at a time).  Each warp then streams whole pages of
+// the range, U vectors per lane ahead, so that an SM reads several pages at
+// once wherever they lie in the pool.  A page id outside the pool sets *bad and
+// that page is not counted.
+template <int DT, int NT>
+__device__ void count_range_paged(uint32_t *col, uint32_t inc, const uint8_t *pool, const PageRef &pr,
+                                  uint64_t a, uint64_t b, int32_t *s_ids, bool *bad) {
+    using C = PlanCfg<DT>;
+    constexpr int U = kPlanUnroll;
+    const int tid = threadIdx.x;
+    const uint64_t pe = pr.page_elems;
+    // whole vectors only; the ragged end (< one vector) is counted below
+    const uint64_t b_vec = a + (b - a) / C::kVecElems * C::kVecElems;
+    for (uint64_t p0 = a / pe; p0 * pe < b_vec; p0 += kPageCache) {
+        const uint64_t lo = max(a, p0 * pe), hi = min(b_vec, (p0 + kPageCache) * pe);
+        const uint32_t npg = uint32_t((hi - 1) / pe - p0 + 1);
+        __syncthreads();  // the previous pass is done with s_ids
+        for (uint32_t i = tid; i < npg; i += NT) s_ids[i] = __ldg(pr.pages + p0 + i);
+        __syncthreads();
+        // warp w takes pages w, w + NW, ... of the pass: every warp streams its own
+        // page, so an SM has NW pages in flight (pages lie anywhere in the pool)
+        constexpr int NW = NT / 32;
+        const int warp = tid >> 5, lane = tid & 31;
+        for (uint32_t j = uint32_t(warp); j < npg; j += NW) {
+            const uint64_t ps = (p0 + j) * pe;
+            const uint64_t x = max(lo, ps), y = min(hi, ps + pe);
+            const int32_t id = s_ids[j];
+            if (id < 0 || uint64_t(id) >= pr.pool_pages) {
+                *bad = true;
+                continue;
+            }
+            const uint4 *src = reinterpret_cast<const uint4 *>(pool + uint64_t(id) * pr.page_bytes +
+                                                                (x - ps) * C::kElemBytes);
+            const uint32_t nvec = uint32_t((y - x) / C::kVecElems);
+            uint4 cur[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t k = uint32_t(lane) + uint32_t(u) * 32;
+                cur[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+            }
+            for (uint32_t base = 0; base < nvec; base += uint32_t(U) * 32) {
+                uint4 nxt[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const uint32_t k = base + uint32_t(U) * 32 + uint32_t(lane) + uint32_t(u) * 32;
+                    nxt[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (base + uint32_t(lane) + uint32_t(u) * 32 < nvec) count_vec<DT, NT>(col, inc, cur[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+            }
+        }
+    }
+    // ragged end (< one vector): thread 0 counts it element by element
+    if (tid == 0) {
+        for (uint64_t i = b_vec; i < b; ++i) {
+            const uint64_t off = elem_offset<C::kElemBytes>(pr, i);
+            if (off == kBadOffset) {
+                *bad = true;
+                continue;
+            }
+            atomicAdd(col + exponent_scalar<DT>(pool + off, 0) * (NT / 2), inc);
+        }
+    }
+}
+
 // Add every column into the global histogram g_hist and clear them.
 template <int DT, int NT>
 __device__ void flush_columns(uint32_t *s_cols, uint32_t *g_hist) {
@@ -190,7 +263,8 @@ __device__ void select_codebook(uint32_t *g_hist, uint32_t *g_ticket, uint64_t n
 template <int DT, int NT, int MAXB>
 __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ PlanParams<MAXB> p) {
     using C = PlanCfg<DT>;
-    extern __shared__ uint32_t s_cols[];  // C::kBins * NT/2 words of two 16-bit counters
+    extern __shared__ uint32_t s_cols[];  // C::kBins * NT/2 words of two 16-bit counters, then page ids
+    int32_t *s_ids = reinterpret_cast<int32_t *>(s_cols + C::kBins * (NT / 2));
     __shared__ uint32_t s_cnt[C::kBins];
     __shared__ uint8_t s_cb[16];
     __shared__ uint32_t s_words[16];
@@ -231,22 +305,19 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
         // sub-ranges short enough that no 16-bit counter can overflow
         constexpr uint64_t kSub = uint64_t(kMaxPerThread / C::kVecElems) * C::kVecElems * NT;
         const PageRef &pr = p.pg[t];
-        for (uint64_t s = a; s < b; s += kSub) {
-            const uint64_t e = min(b, s + kSub);
+        // Paged ranges are counted page by page per warp, so one lane may see up to
+        // range / NT + 1.25 page / 32 elements: half-size sub-ranges keep that below
+        // 65535 for pages of up to 2^18 elements (the host's limit).
+        constexpr uint64_t kSubPaged = uint64_t(kMaxPerThread / 2) * NT;
+        const uint64_t sub = pr.pages ? kSubPaged : kSub;
+        for (uint64_t s = a; s < b; s += sub) {
+            const uint64_t e = min(b, s + sub);
             if (!pr.pages) {
                 count_range<DT, NT>(col, inc, p.in[t], s, e);
             } else {
-                // a paged tensor: count each page's piece from its own address
-                for (uint64_t x = s; x < e;) {
-                    const uint64_t y = min(e, (x / pr.page_elems + 1) * pr.page_elems);
-                    const uint64_t off = elem_offset<C::kElemBytes>(pr, x);
-                    if (off == kBadOffset) {
-                        if (tid == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, uint32_t(t));
-                    } else {
-                        count_range<DT, NT>(col, inc, p.in[t] + off, 0, y - x);
-                    }
-                    x = y;
-                }
+                bool bad = false;
+                count_range_paged<DT, NT>(col, inc, p.in[t], pr, s, e, s_ids, &bad);
+                if (bad) set_error(p.ctl, SZ_ERR_INVALID_ARG, uint32_t(t));
             }
             flush_columns<DT, NT>(s_cols, g_hist);
         }
@@ -286,10 +357,14 @@ sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
         p.item_begin[t + 1] = p.item_begin[t] + cdiv(a.n[t], C::kItemElems);
     }
     p.total_items = p.item_begin[a.T];
-    const size_t smem = size_t(C::kBins) * (NT / 2) * 4;
+    bool any_paged = false;
+    for (int t = 0; t < a.T; ++t) any_paged = any_paged || (a.paged && a.paged[t].pages && a.n[t]);
+    const size_t smem = size_t(C::kBins) * (NT / 2) * 4 + (any_paged ? size_t(kPageCache) * 4 : 0);
     auto kern = plan_kernel<DT, NT, MAXB>;
+    // the kernel's shared-memory limit is set once, for the larger (paged) need
+    const size_t smem_max = size_t(C::kBins) * (NT / 2) * 4 + size_t(kPageCache) * 4;
     static std::atomic<int> cache[kMaxDevices];
-    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
+    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem_max, cache);
     if (per_sm < 1) return SZ_ERR_CUDA;
     uint64_t grid = uint64_t(a.num_sms) * per_sm;
     if (p.total_items < grid) grid = p.total_items;

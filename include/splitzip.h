@@ -106,7 +106,8 @@ typedef struct {
  *               that page is neither read nor written
  *   page_bytes  bytes from one page to the next, a multiple of 16 and at least
  *               page_elems * elem_bytes
- *   page_elems  elements of this tensor per page, a multiple of 1024 */
+ *   page_elems  elements of this tensor per page, a multiple of 1024, at most
+ *               2^18 */
 typedef struct {
     const void *pool;
     const int32_t *pages;

@@ -154,7 +154,7 @@ def test_paged_host_checks():
     ws = m.new_workspace(0, [4096])
     plans = m.new_plans(1)
     for kw in (dict(page_elems=1000), dict(page_elems=1024, page_bytes=2 * 1024 + 8),
-               dict(page_elems=1024, page_bytes=1024)):
+               dict(page_elems=1024, page_bytes=1024), dict(page_elems=(1 << 18) + 1024)):
         d = m.paged(0, pool, ids, **kw)
         with pytest.raises(m.SplitZipError) as e:
             m.sz_plan_paged_batched(0, [d], [4096], ws, plans)
@@ -193,3 +193,29 @@ def test_paged_batch_and_reuse():
     assert m.sz_last_device_status(ws) == 0
     for raw, out, t in zip(raws, outs, totals.cpu().tolist()):
         assert np.array_equal(out[:t].cpu().numpy(), oracle.encode_codebook(1, raw, cb))
+
+
+def test_largest_pages():
+    """Pages of 2^18 elements (the limit): the histogram's per-lane counts stay in range."""
+    m = sz()
+    rng = np.random.default_rng(31)
+    pe = 1 << 18
+    sizes = [3 * pe + 4100, 70000]
+    raws = [oracle_pins._kvlike(rng, n, 0) for n in sizes]
+    # one exponent dominates, so single counters grow as fast as possible
+    for r in raws:
+        w = r.view("<u2")
+        w[rng.random(w.size) < 0.9] = 0x3F80
+    pool_h, tables_h, page_bytes, pool_pages = build_pool(rng, 0, raws, pe, 0)
+    pool = torch.from_numpy(pool_h).cuda()
+    tables = [torch.from_numpy(t).cuda() for t in tables_h]
+    srcs = [m.paged(0, pool, t, pe, page_bytes, pool_pages) for t in tables]
+    ws = m.new_workspace(0, sizes)
+    plans = m.new_plans(2)
+    m.sz_plan_paged_batched(0, srcs, sizes, ws, plans)
+    outs = [torch.zeros(m.sz_max_compressed_size(0, n), dtype=torch.uint8, device="cuda") for n in sizes]
+    m.sz_encode_paged_batched(0, plans, srcs, sizes, outs, ws)
+    assert m.sz_last_device_status(ws) == 0
+    for raw, out in zip(raws, outs):
+        ref = oracle.encode(0, raw)
+        assert np.array_equal(out[: ref.size].cpu().numpy(), ref)
