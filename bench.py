@@ -86,12 +86,14 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("sz_common.cuh", "sz_plan.cu", "sz_encode.cu", "sz_decode.cu")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources and the C-ABI header (which kernels a profile describes)."""
-    import glob
+    """Hash of the device-code sources (which kernels a profile describes); host-only
+    files (the C-ABI layer, the header) do not change it."""
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", "*")))
-    files.append(os.path.join(ROOT, "include", "splitzip.h"))
+    files = [os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", f) for f in KERNEL_SOURCES]
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())

@@ -236,6 +236,33 @@ __device__ __forceinline__ void patch(uint32_t (&o)[4], uint32_t j, uint32_t e) 
     o[3] += (k == 3) ? add : 0u;
 }
 
+// Escapes of one step by the general path: warp prefix of the per-lane counts c
+// and a per-lane loop over the escape flags m (bit 4j: element j), patching
+// each escape's exponent into o.
+template <int DT, typename M>
+__device__ __forceinline__ void patch_escapes(uint32_t (&o)[4], M m, uint32_t c, uint32_t &running,
+                                              uint32_t esc_reg, const uint8_t *esc_g, uint32_t cnt, bool &bad) {
+    uint32_t tot;
+    const uint32_t prefix = warp_exclusive_prefix(c, &tot);
+    const uint32_t maxc = __reduce_max_sync(0xffffffffu, c);
+    M mm = m;
+    for (uint32_t i = 0; i < maxc; ++i) {
+        const uint32_t r = running + prefix + i;
+        const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
+        if (i < c) {
+            // element, in element order
+            const uint32_t j = uint32_t((DT == SZ_BF16) ? __ffs(uint32_t(mm)) - 1 : __ffsll(uint64_t(mm)) - 1) >> 2;
+            mm &= mm - 1;
+            uint32_t e = 0;
+            if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
+            else bad = true;
+            if (DT == SZ_FP8_E5M2 && e >= 32u) bad = true;
+            patch<DT>(o, j, e & (Dt<DT>::kBins - 1));
+        }
+    }
+    running += tot;
+}
+
 // Decode one step.  running: escapes of the block before this step (updated);
 // esc_reg: lane i holds the block's escape i (i < 32); esc_g: the block's
 // escapes in global memory; cnt: escapes the offsets table gives the block.
@@ -244,8 +271,6 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
                                             uint8_t *dst, int valid, uint32_t &running, uint32_t esc_reg,
                                             const uint8_t *esc_g, uint32_t cnt, bool &bad, bool store = true) {
     uint32_t o[4];
-    // escape flags of this lane's elements: bit 4j for element j
-    typename std::conditional<DT == SZ_BF16, uint32_t, uint64_t>::type m;
     if constexpr (DT == SZ_BF16) {
         const uint32_t cw = f.c0;
 #pragma unroll
@@ -254,8 +279,54 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
             const uint32_t x = __byte_perm((k < 2) ? f.a : f.b, 0, (k & 1) ? 0x4342 : 0x4140);
             o[k] = x + (x & 0x00800080u) * 0xFFu + (e2 << 7);
         }
-        m = escape_nibbles(cw);
+        const uint32_t m = escape_nibbles(cw);  // bit 4j: element j is escaped
+        const uint32_t c = __popc(m);
+        const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+        if (any == 0) {
+            // no escape in this step
+        } else if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+            // at most one escape per lane: its rank counts the lanes before it that have one
+            const uint32_t lane = threadIdx.x & 31;
+            const uint32_t r = running + __popc(any & ((1u << lane) - 1u));
+            const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
+            if (c) {
+                const uint32_t j = uint32_t(__ffs(m) - 1) >> 2;
+                uint32_t e = 0;
+                if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
+                else bad = true;
+                patch<DT>(o, j, e & 0xFFu);
+            }
+            running += __popc(any);
+        } else {
+            patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
+        }
     } else {
+        // Escapes first.  With at most one escape per lane (the usual case) its
+        // exponent takes the place of code 15's byte in this lane's table, so the
+        // lookups below produce it directly; otherwise (general) the escapes are
+        // patched in afterwards.
+        const uint64_t m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
+        const uint32_t c = __popcll(m);
+        const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+        uint32_t xt3 = xt[3];
+        bool general = false;
+        if (any != 0) {
+            if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+                const uint32_t lane = threadIdx.x & 31;
+                const uint32_t r = running + __popc(any & ((1u << lane) - 1u));
+                const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
+                if (c) {
+                    uint32_t e = 0;
+                    if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
+                    else bad = true;
+                    if (e >= 32u) bad = true;
+                    xt3 = (xt3 & 0x00FFFFFFu) | ((e & 31u) << 26);  // table byte 15 = exponent x 4 (< 128)
+                }
+                running += __popc(any);
+            } else {
+                general = true;
+            }
+        }
         // four codes per word select their exponents from the register table:
         // codes 0-7 from bytes 0-7, codes 8-15 from bytes 8-15 (selector with
         // the top bit flipped, so each half reads zero for the other's codes)
@@ -266,7 +337,7 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
         for (int k = 0; k < 4; ++k) {
             const uint32_t cw = (k < 2) ? f.c0 : f.c1, cx = (k < 2) ? x0 : x1;
             const uint32_t sl = (k & 1) ? (cw >> 16) : cw, sh = (k & 1) ? (cx >> 16) : cx;
-            const uint32_t e_lo = prmt(xt[0], xt[1], sl), e_hi = prmt(xt[2], xt[3], sh);
+            const uint32_t e_lo = prmt(xt[0], xt[1], sl), e_hi = prmt(xt[2], xt3, sh);
             // Spreads by multiplication (the partial products never overlap a
             // kept bit): sign bits 4k..4k+3 of plane a to bit 7 of bytes 0-3,
             // the four 2-bit mantissas of byte k of plane b to bits 0-1.
@@ -276,46 +347,7 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
                                 prmt(od, 0u, 0x4440u + uint32_t(k)) * 0x40040u;
             o[k] = ((sg & 0x80808080u) | e_hi) | ((mn & 0x03030303u) | e_lo);
         }
-        m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
-    }
-    const uint32_t c = (DT == SZ_BF16) ? uint32_t(__popc(uint32_t(m))) : uint32_t(__popcll(uint64_t(m)));
-    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
-    if (any == 0) {
-        // no escape in this step
-    } else if (__ballot_sync(0xffffffffu, c > 1) == 0) {
-        // at most one escape per lane: its rank counts the lanes before it that have one
-        const uint32_t lane = threadIdx.x & 31;
-        const uint32_t r = running + __popc(any & ((1u << lane) - 1u));
-        const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
-        if (c) {
-            const uint32_t j = uint32_t((DT == SZ_BF16) ? __ffs(uint32_t(m)) - 1 : __ffsll(uint64_t(m)) - 1) >> 2;
-            uint32_t e = 0;
-            if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
-            else bad = true;
-            if (DT == SZ_FP8_E5M2 && e >= 32u) bad = true;
-            patch<DT>(o, j, e & (Dt<DT>::kBins - 1));
-        }
-        running += __popc(any);
-    } else {
-        uint32_t tot;
-        const uint32_t prefix = warp_exclusive_prefix(c, &tot);
-        const uint32_t maxc = __reduce_max_sync(0xffffffffu, c);
-        auto mm = m;
-        for (uint32_t i = 0; i < maxc; ++i) {
-            const uint32_t r = running + prefix + i;
-            const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
-            if (i < c) {
-                // element, in element order
-                const uint32_t j = uint32_t((DT == SZ_BF16) ? __ffs(uint32_t(mm)) - 1 : __ffsll(uint64_t(mm)) - 1) >> 2;
-                mm &= mm - 1;
-                uint32_t e = 0;
-                if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
-                else bad = true;
-                if (DT == SZ_FP8_E5M2 && e >= 32u) bad = true;
-                patch<DT>(o, j, e & (Dt<DT>::kBins - 1));
-            }
-        }
-        running += tot;
+        if (general) patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
     }
     if (CHECKED && !store) {
         // an output page outside the pool: nothing is written
