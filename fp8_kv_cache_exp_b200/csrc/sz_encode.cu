@@ -31,19 +31,19 @@ constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
 constexpr int kChunkBlocks = 8;                       // a warp's unit of work: 8 consecutive blocks
 constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per chunk (two chunks)
-constexpr int kRing = 3;                              // quarter-block input stages per warp
-constexpr uint32_t kQuarterBytes = 2048;              // largest quarter block (BF16)
+constexpr int kRing = 3;                              // input-unit stages per warp
+constexpr uint32_t kUnitBytes = 2048;                 // one input unit: a quarter block (BF16) or half a block (E5M2)
 constexpr int kLookbackPerLane = 4;                   // status words per lane per step
 constexpr uint64_t kLookbackLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr uint64_t kWaitLimitNs = 1000000000ull;      // bulk-copy wait limit
 constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate published
 constexpr unsigned long long kFlagInc = 2ull << 32;   // inclusive prefix published
 
-// Each warp works alone: its own input ring (bulk copies of quarter blocks),
+// Each warp works alone: its own input ring (bulk copies of 2 KB units),
 // plan header, exponent -> code table, and two escape stages (the chunk being
 // coded and one whose offset is still being looked up).
 struct alignas(128) WarpShared {
-    uint8_t ring[kRing][kQuarterBytes];
+    uint8_t ring[kRing][kUnitBytes];
     uint64_t bar[kRing];
     uint32_t hdr[16];
     uint32_t blk_off[2][kChunkBlocks];  // escapes before each block, within the chunk
@@ -463,8 +463,8 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     return running;
 }
 
-// The warp's input ring: units are quarter blocks of the chunk being coded,
-// stage = unit % kRing; quarters of a partial (last) block are not copied and
+// The warp's input ring: units (Units below) of the chunk being coded,
+// stage = unit % kRing; units of a partial (last) block are not copied and
 // are read from global memory instead.
 struct RingState {
     uint32_t issued;  // bit s: stage s holds a copy not yet waited for
@@ -472,20 +472,32 @@ struct RingState {
     uint32_t vi, vc;  // units issued / consumed
 };
 
-template <int DT>
+// Units per 4096-element block of the input ring: 2 KB units, i.e. quarter
+// blocks for BF16 and half blocks for E5M2 -- but quarter blocks for paged E5M2
+// input, whose pages are only known to hold multiples of 1024 elements.
+template <int DT, bool PAGED>
+struct Units {
+    static constexpr int kPerBlock = (DT == SZ_BF16 || PAGED) ? 4 : 2;
+    static constexpr uint32_t kElems = kBlock / kPerBlock;
+    static constexpr uint32_t kBytes = kElems * Dt<DT>::kElemBytes;
+    static_assert(kBytes <= kUnitBytes, "a unit must fit a ring stage");
+};
+
+template <int DT, bool PAGED>
 __device__ __forceinline__ void ring_issue(WarpShared &W, RingState &R, const uint8_t *in, uint64_t n,
                                            uint64_t b0, uint32_t x, bool paged, uint64_t paged_off, uint32_t *ctl) {
-    constexpr uint32_t kQB = kBlock / 4 * Dt<DT>::kElemBytes;  // bytes of a quarter block
+    using U = Units<DT, PAGED>;
     const int st = int(R.vi % kRing);
-    const uint64_t blk = b0 + x / 4;
+    const uint64_t blk = b0 + x / U::kPerBlock;
     if ((blk + 1) * kBlock <= n) {
-        // byte offset of the quarter from the input base (paged: looked up by the caller)
-        const uint64_t off = paged ? paged_off : (blk * kBlock + (x % 4) * (kBlock / 4)) * Dt<DT>::kElemBytes;
+        // byte offset of the unit from the input base (paged: looked up by the caller)
+        const uint64_t off = paged ? paged_off
+                                   : (blk * kBlock + (x % U::kPerBlock) * U::kElems) * Dt<DT>::kElemBytes;
         if (off != kBadOffset) {
             if ((threadIdx.x & 31) == 0) {
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&W.bar[st], kQB);
-                bulk_g2s(W.ring[st], in + off, kQB, &W.bar[st]);
+                mbar_arrive_expect_tx(&W.bar[st], U::kBytes);
+                bulk_g2s(W.ring[st], in + off, U::kBytes, &W.bar[st]);
             }
             R.issued |= 1u << st;
         } else if ((threadIdx.x & 31) == 0) {
@@ -574,18 +586,19 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
     const Layout L = stream_layout(DT, n, p.reuse ? 0 : H.E);  // section starts do not depend on E
 
     using G = Geo<DT>;
-    constexpr int QIT = G::IT / 4;  // steps per quarter block
+    using UN = Units<DT, PAGED>;
+    constexpr int QIT = G::IT / UN::kPerBlock;  // steps per unit
     const uint32_t lut = lut_addr(W), stage = smem_u32(W.esc[slot]);
-    const uint32_t nunits = 4u * uint32_t(nbk);
+    const uint32_t nunits = uint32_t(UN::kPerBlock) * uint32_t(nbk);
     // paged input: lane x looks up where unit x (a quarter block) of the chunk lives
     const PageRef &pr = p.pg[g.t];
     const bool paged = PAGED && pr.pages != nullptr;
     uint64_t unit_off = 0;
-    if (paged && uint32_t(lane) < nunits && b0 * kBlock + uint64_t(lane) * (kBlock / 4) < n)
-        unit_off = elem_offset<Dt<DT>::kElemBytes>(pr, b0 * kBlock + uint64_t(lane) * (kBlock / 4));
+    if (paged && uint32_t(lane) < nunits && b0 * kBlock + uint64_t(lane) * UN::kElems < n)
+        unit_off = elem_offset<Dt<DT>::kElemBytes>(pr, b0 * kBlock + uint64_t(lane) * UN::kElems);
     auto issue = [&](uint32_t x) {
         const uint64_t off = paged ? __shfl_sync(0xffffffffu, unit_off, int(x)) : 0ull;
-        ring_issue<DT>(W, R, in, n, b0, x, paged, off, p.ctl);
+        ring_issue<DT, PAGED>(W, R, in, n, b0, x, paged, off, p.ctl);
     };
     uint32_t next_x = 0;
     for (; next_x < uint32_t(kRing - 1) && next_x < nunits; ++next_x) issue(next_x);
@@ -603,7 +616,7 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
         };
         uint32_t blk_run = 0;
 #pragma unroll 1
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < UN::kPerBlock; ++qq) {
             if (next_x < nunits) issue(next_x++);
             int st;
             *lost = !ring_take(W, R, &st) || *lost;
