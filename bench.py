@@ -350,7 +350,8 @@ def run_ours(args, rank, world, device):
         k["gbs"] = k["bytes"] / (k["ms"] * 1e-3) / 1e9
         k["frac"] = k["gbs"] / peak
     dom = max(kern, key=lambda k: kern[k]["ms"])
-    traffic = profiled_traffic(dom + "_kernel", wl.name) if world == 1 else None
+    key = wl.name + ("+paged%d" % args.paged if args.paged else "")
+    traffic = profiled_traffic(dom + "_kernel", key) if world == 1 and not args.layers else None
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(kern[dom]["gbs"], 1), "peak": peak,
             "unit": "GB/s", "frac": round(kern[dom]["frac"], 4),
             "traffic": traffic, "algorithmic_bytes": kern[dom]["bytes"],
