@@ -383,6 +383,78 @@ def run_ours(args, rank, world, device):
     return res, wl
 
 
+def run_transfer(args, wl, device, res):
+    """Layer-pipelined transfer (fp8_kv_cache_exp_b200.transfer): per layer, plan +
+    encode on the source, decode on the destination from the source's streams.
+    One GPU: source and destination are the same device (the link is not crossed);
+    the pipeline's device time is measured, and the transfer over a link of speed B
+    is modelled from the measured per-layer codec times (FastKVComp page, Equation 1
+    for the break-even)."""
+    from fp8_kv_cache_exp_b200.transfer import LayerPipeline, break_even_gbs, pipelined_seconds
+    layers = [[wl.xs[2 * i], wl.xs[2 * i + 1]] for i in range(len(wl.xs) // 2)]
+    pipe = LayerPipeline(layers, device)
+    for _ in range(args.warmup):
+        pipe.run()
+    pipe.synchronize()
+    # per-layer stage times, from one instrumented pass (events around each call)
+    enc_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    import fp8_kv_cache_exp_b200 as sz
+    for i, (b, outs, dec, ws) in enumerate(zip(pipe.batches, pipe.outs, pipe.decoded, pipe.ws_dst)):
+        with torch.cuda.stream(pipe.s_src):
+            enc_ev[i][0].record(pipe.s_src)
+            b.plan(stream=pipe.s_src)
+            b.encode(stream=pipe.s_src)
+            enc_ev[i][1].record(pipe.s_src)
+        pipe.s_dst.wait_stream(pipe.s_src)
+        with torch.cuda.stream(pipe.s_dst):
+            dec_ev[i][0].record(pipe.s_dst)
+            sz.sz_decode_batched(wl.dtype, outs, dec, ws, stream=pipe.s_dst)
+            dec_ev[i][1].record(pipe.s_dst)
+        pipe.s_src.wait_stream(pipe.s_dst)
+    pipe.synchronize()
+    t_enc = [a.elapsed_time(b) * 1e-3 for a, b in enc_ev]
+    t_dec = [a.elapsed_time(b) * 1e-3 for a, b in dec_ev]
+    # the pipelined run itself
+    K = args.steps
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(pipe.s_src)
+    for _ in range(K):
+        pipe.run()
+    pipe.s_src.wait_stream(pipe.s_dst)
+    stop.record(pipe.s_src)
+    pipe.synchronize()
+    ms = start.elapsed_time(stop) / K
+    for src, out in zip(layers, pipe.decoded):
+        for x, y in zip(src, out):
+            if not torch.equal(x.view(torch.uint8), y.view(torch.uint8)):
+                raise RuntimeError("transfer round trip mismatch")
+    ratio = res["ratio"]
+    S = float(wl.raw_bytes)
+    layer_bytes = [float(x.numel() * x.element_size() + y.numel() * y.element_size()) for x, y in layers]
+    codec_s = sum(t_enc) + sum(t_dec)
+    links = {}
+    for name, gbs in (("RoCE 4x200 Gb/s (the SplitZip setup)", 100.0), ("NVLink 5, 900 GB/s nominal", 900.0)):
+        B = gbs * 1e9
+        raw_s = S / B
+        serial_s = codec_s + S / (ratio * B)
+        piped_s = pipelined_seconds([(te, lb / (ratio * B), td) for te, td, lb in zip(t_enc, t_dec, layer_bytes)])
+        links[name] = {"link_gbs": gbs, "raw_ms": round(raw_s * 1e3, 4), "compressed_serial_ms": round(serial_s * 1e3, 4),
+                       "compressed_pipelined_ms": round(piped_s * 1e3, 4),
+                       "speedup_pipelined": round(raw_s / piped_s, 3)}
+    return {
+        "pipeline_ms_per_step": round(ms, 4),
+        "pipeline_gbs": round(S / (ms * 1e-3) / 1e9, 1),
+        "devices": "one GPU: source and destination are the same device (loopback)",
+        "layers": len(layers),
+        "encode_ms_per_layer": round(1e3 * sum(t_enc) / len(layers), 4),
+        "decode_ms_per_layer": round(1e3 * sum(t_dec) / len(layers), 4),
+        "break_even_gbs_serial": round(break_even_gbs(S, ratio, codec_s), 1),
+        "model": links,
+        "model_note": "link times are modelled from the measured per-layer codec times; the link is not measured",
+    }
+
+
 def run_e2e(args, wl, device):
     """Same metric through the C ABI with host buffers: pinned H2D of the raw batch,
     plan + encode + decode, D2H of the decoded batch, all inside the timed region."""
@@ -535,6 +607,8 @@ def main():
                     help="codebook reuse: plan once, then every step is encode with those codebooks + decode")
     ap.add_argument("--paged", type=int, default=0, metavar="TOKENS",
                     help="hold the tensors in pages of TOKENS tokens (paged KV), in random page order")
+    ap.add_argument("--transfer", action="store_true",
+                    help="also run the layer-pipelined transfer (encode on the source, decode on the destination)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -564,6 +638,8 @@ def main():
                 max_over_ranks(e2e["ms_per_step"], world, device) * 1e-3) / 1e9
             e2e["value"] = round(e2e_val, 2)
             res["e2e"] = e2e
+        if args.transfer:
+            res["transfer"] = run_transfer(args, wl, device, res)
         if rank == 0 and world == 1 and args.cpu_baseline_seconds > 0:
             res["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload][0], args.cpu_baseline_seconds)
         if rank == 0:

@@ -18,7 +18,8 @@ __all__ = [
     "sz_max_compressed_size", "sz_workspace_init", "sz_plan", "sz_plan_batched",
     "sz_compressed_size", "sz_compressed_sizes", "sz_encode", "sz_encode_batched",
     "sz_encode_reuse", "sz_encode_reuse_batched", "sz_plan_paged_batched", "sz_encode_paged_batched",
-    "sz_decode_paged_batched", "sz_encode_reuse_paged_batched", "sz_paged_t", "paged", "sz_decode",
+    "sz_decode_paged_batched", "sz_encode_reuse_paged_batched", "sz_paged_t", "paged", "sz_enable_peer_access",
+    "sz_decode",
     "sz_decode_batched", "sz_last_device_status", "sz_encode_noalloc", "dtype_of", "elem_bytes", "numel_of",
     "new_workspace", "new_plans", "Batch",
 ]
@@ -80,6 +81,7 @@ def _load():
         "sz_decode": (i32, [i32, vp, sz, vp, u64, vp, sz, vp]),
         "sz_decode_batched": (i32, [i32, i32, pvp, psz, pvp, pu64, vp, sz, vp]),
         "sz_last_device_status": (i32, [vp, vp]),
+        "sz_enable_peer_access": (i32, [i32, i32]),
         "sz_encode_noalloc": (i32, [i32, vp, vp, u64, vp, sz, vp, vp]),
     }
     for name, (res, args) in sigs.items():
@@ -419,6 +421,11 @@ class Batch:
             return
         _check(lib.sz_decode_batched(self.dtype, self.T, self._out, self._cb, self._dec, self._dn,
                                      self._ws, self._wsb, _stream(stream)), "sz_decode_batched")
+
+
+def sz_enable_peer_access(device: int, peer: int):
+    """Let this library's kernels on `device` read `peer`'s memory (see the C header)."""
+    _check(lib.sz_enable_peer_access(int(device), int(peer)), "sz_enable_peer_access")
 
 
 def sz_last_device_status(ws: torch.Tensor, stream=None) -> int:

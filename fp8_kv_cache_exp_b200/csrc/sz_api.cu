@@ -243,6 +243,23 @@ sz_status sz_decode(sz_dtype dtype, const void *d_comp, size_t comp_bytes, void 
     return sz_decode_batched(dtype, 1, comp, &comp_bytes, out, &n, d_ws, ws_bytes, stream);
 }
 
+sz_status sz_enable_peer_access(int device, int peer) {
+    if (device < 0 || peer < 0) return SZ_ERR_INVALID_ARG;
+    if (device == peer) return SZ_OK;
+    int prev = 0, can = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess) return SZ_ERR_CUDA;
+    if (cudaDeviceCanAccessPeer(&can, device, peer) != cudaSuccess || !can) return SZ_ERR_CUDA;
+    if (cudaSetDevice(device) != cudaSuccess) return SZ_ERR_CUDA;
+    cudaError_t e = cudaDeviceEnablePeerAccess(peer, 0);
+    if (e == cudaErrorPeerAccessAlreadyEnabled) {
+        cudaGetLastError();  // clear the sticky-free "already enabled" status
+        e = cudaSuccess;
+    }
+    const bool ok = e == cudaSuccess;
+    if (cudaSetDevice(prev) != cudaSuccess) return SZ_ERR_CUDA;
+    return ok ? SZ_OK : SZ_ERR_CUDA;
+}
+
 sz_status sz_last_device_status(void *d_ws, cudaStream_t stream) {
     if (!d_ws || !aligned(d_ws, 8)) return SZ_ERR_INVALID_ARG;
     uint32_t err[2] = {0, 0};

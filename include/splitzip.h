@@ -230,6 +230,16 @@ sz_status sz_encode_reuse_paged_batched(sz_dtype dtype, int T, const sz_plan_t *
                                         const size_t *out_cap, uint64_t *d_totals, void *d_ws, size_t ws_bytes,
                                         cudaStream_t stream);
 
+/* Let kernels on CUDA device `device` read the memory of device `peer`
+ * directly (peer access over NVLink).  After it, sz_decode* on `device` may be
+ * given streams that live on `peer`: the decode kernel then pulls each
+ * stream's bytes across the link itself, with the same 1-D bulk copies it uses
+ * for local streams (no multicast), so the transfer overlaps the decoding
+ * tile by tile and the stream never lands in `device`'s memory.
+ * SZ_OK if access is enabled (or already was; device == peer needs nothing),
+ * SZ_ERR_CUDA if the two devices cannot reach each other. */
+sz_status sz_enable_peer_access(int device, int peer);
+
 /* Decode a stream of comp_bytes bytes holding n elements of dtype into d_out
  * (BF16: 2n bytes, E5M2: n bytes); the result is bitwise identical to the
  * encoded input (project page, FAQ "Is SplitZip lossy?").  A stream that fails
