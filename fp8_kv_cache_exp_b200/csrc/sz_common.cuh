@@ -157,9 +157,10 @@ struct PlanParams {
     PageRef pg[MAXB];
 };
 
-// Encode and decode work in chunks: up to kMaxChunkBlocks consecutive
-// 4096-element blocks of one tensor.  One look-back status word per chunk.
-constexpr int kMaxChunkLog2 = 4;
+// Encode works in chunks of 1 << chunk_log2 consecutive 4096-element blocks of
+// one tensor (chunk_log2 <= kMaxChunkLog2).  One look-back status word per
+// chunk; the workspace holds one per block, enough for any chunk size.
+constexpr int kMaxChunkLog2 = 3;
 constexpr int kMaxChunkBlocks = 1 << kMaxChunkLog2;
 
 template <int MAXB>
@@ -198,10 +199,14 @@ struct DecodeParams {
 };
 
 // Blocks per chunk for a launch: the largest power of two (<= kMaxChunkBlocks)
-// that still leaves at least two chunks per resident CTA.
-inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_ctas) {
+// that still gives at least one chunk per two resident warps.  Every chunk
+// costs a claim, a look-back and a ring restart, so chunks stay as long as the
+// launch allows: a large batch keeps 8-block chunks, one layer's K and V
+// (4096 BF16 or 8192 E5M2 blocks) gets 2- or 4-block chunks and still spreads
+// over every SM (measured best for both).
+inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_warps) {
     int lg = kMaxChunkLog2;
-    while (lg > 0 && (total_blocks >> lg) < 2 * resident_ctas) --lg;
+    while (lg > 0 && (total_blocks >> lg) < resident_warps / 2) --lg;
     return lg;
 }
 

@@ -2,22 +2,26 @@
 //
 // SplitZip project page, Abstract: sign and mantissa bits are kept exactly,
 // frequent exponents get fixed 4-bit codes, rare exponents go to a sparse
-// escape stream.  Persistent CTAs take chunks (up to 16 consecutive
-// 4096-element blocks of one tensor) in launch order from an atomic counter:
-//   1. each block: 16-byte loads (the next block prefetched), exponent -> code
-//      through a 256-entry shared table built from the plan's codebook,
-//      sign|mantissa bytes (BF16) or sign bits + 2-bit mantissas (E5M2) and
-//      4-bit codes written with coalesced 2-8 byte stores;
-//   2. escapes of each block ranked by a CTA prefix sum and staged in shared
-//      memory in element order, with the block's offset within the chunk;
-//   3. the chunk's escape offset found by a single-pass decoupled look-back
-//      over the chunks of its tensor: every chunk with a lower id is already
-//      claimed by a running CTA, a 128-chunk window is read per step, and the
-//      wait is bounded (SZ_ERR_TIMEOUT instead of a hang);
-//   4. the chunk's entries of the offsets table and its staged escapes written
-//      contiguously (a chunk whose escapes overflow the stage re-reads its
-//      input and writes them directly); the tensor's last chunk also writes
-//      the header, offsets[nb] and the zero padding between sections.
+// escape stream.  Persistent CTAs of 8 independent warps (no CTA barrier on the
+// path).  Each warp takes chunks -- 1 to 8 consecutive 4096-element blocks of
+// one tensor, short chunks for small batches -- in launch order from an atomic
+// counter:
+//   1. the chunk's input arrives by 1-D bulk copies of 2 KB units into the
+//      warp's 3-stage shared-memory ring (bounded mbarrier waits);
+//   2. per step a lane codes 8 (BF16) or 16 (E5M2) elements from one 16-byte
+//      shared load: exponent -> code through a 256-byte table whose entry
+//      address one prmt forms, sign|mantissa planes and 4-bit codes written
+//      with coalesced stores; escapes ranked by ballots (a fast path when no
+//      lane has two) and staged in element order in the warp's stage;
+//   3. the chunk's escape offset comes from a single-pass decoupled look-back
+//      over the chunks of its tensor (128 predecessors per step, resumable; a
+//      chunk whose predecessors have not yet published is finished between the
+//      blocks of the warp's next chunk; every wait is bounded: SZ_ERR_TIMEOUT
+//      instead of a hang);
+//   4. the chunk's offsets-table entries and escapes are written contiguously
+//      (a chunk whose escapes overflow the stage re-codes its input and writes
+//      them directly); the tensor's last chunk writes the header, offsets[nb]
+//      and the zero padding.
 #include <type_traits>
 
 #include "sz_common.cuh"
@@ -29,7 +33,7 @@ namespace {
 
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
-constexpr int kChunkBlocks = 8;                       // a warp's unit of work: 8 consecutive blocks
+constexpr int kChunkBlocks = kMaxChunkBlocks;         // a warp's unit of work: up to 8 consecutive blocks
 constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per chunk (two chunks)
 constexpr int kRing = 3;                              // input-unit stages per warp
 constexpr uint32_t kUnitBytes = 2048;                 // one input unit: a quarter block (BF16) or half a block (E5M2)
@@ -549,15 +553,18 @@ struct ChunkGeo {
     int nbk;
 };
 
-template <int MAXB>
+// LG: blocks per chunk as a log2 fixed at compile time (the full-size chunk of
+// large batches), or -1 to read it from the launch (small batches).
+template <int MAXB, int LG>
 __device__ __forceinline__ ChunkGeo chunk_geo(const EncodeParams<MAXB> &p, uint32_t job) {
+    const int lg = LG >= 0 ? LG : p.chunk_log2;
     ChunkGeo g;
     g.t = find_tensor<uint32_t, MAXB>(p.chunk_begin, p.T, job);
     g.chunk = job - p.chunk_begin[g.t];
     g.n = p.n[g.t];
     g.nb = cdiv(g.n, kBlock);
-    g.b0 = uint64_t(g.chunk) * kChunkBlocks;
-    g.nbk = int(min(uint64_t(kChunkBlocks), g.nb - g.b0));
+    g.b0 = uint64_t(g.chunk) << lg;
+    g.nbk = int(min(uint64_t(1) << lg, g.nb - g.b0));
     return g;
 }
 
@@ -730,7 +737,7 @@ __device__ __forceinline__ unsigned long long *chunk_status(const EncodeParams<M
     return p.status + p.chunk_begin[t];
 }
 
-template <int DT, int MAXB, bool PAGED>
+template <int DT, int MAXB, bool PAGED, int LG>
 __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     extern __shared__ __align__(128) uint8_t s_raw[];
     WarpShared *s_warp = reinterpret_cast<WarpShared *>(s_raw);
@@ -753,7 +760,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
     // finish the pending chunk once its look-back is done (blocking or not)
     auto settle = [&](bool block) {
         if (!pend.valid) return;
-        const ChunkGeo pg = chunk_geo<MAXB>(p, pend.job);
+        const ChunkGeo pg = chunk_geo<MAXB, LG>(p, pend.job);
         if (lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, block)) {
             finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, pend.lb, W);
             pend.valid = false;
@@ -769,7 +776,7 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
             encode_empty<DT, MAXB>(p, p.empty[job - p.total_chunks], W, plan_tensor);
             continue;
         }
-        const ChunkGeo g = chunk_geo<MAXB>(p, job);
+        const ChunkGeo g = chunk_geo<MAXB, LG>(p, job);
         const int slot = pend.valid ? (pend.slot ^ 1) : 0;
         bool lost = false;
         const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost,
@@ -806,10 +813,14 @@ __global__ void __launch_bounds__(NT, 3) encode_kernel(const __grid_constant__ E
 
 template <int DT, int MAXB, bool PAGED>
 sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
-    auto kern = encode_kernel<DT, MAXB, PAGED>;
+    // Full-size chunks (large batches) run an instantiation with the chunk size
+    // fixed at compile time; shorter chunks read it from the launch.  Both are
+    // capped for 3 CTAs per SM and use the same shared memory.
+    auto kern_full = encode_kernel<DT, MAXB, PAGED, kMaxChunkLog2>;
+    auto kern_any = encode_kernel<DT, MAXB, PAGED, -1>;
     const size_t smem = sizeof(WarpShared) * NW;
-    static std::atomic<int> cache[kMaxDevices];
-    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
+    static std::atomic<int> cache_full[kMaxDevices], cache_any[kMaxDevices];
+    const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern_full), NT, smem, cache_full);
     if (per_sm < 1) return SZ_ERR_CUDA;
     const uint64_t resident = uint64_t(a.num_sms) * per_sm;
     EncodeParams<MAXB> p;
@@ -821,7 +832,9 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     for (int t = 0; t < a.T; ++t) p.pg[t] = page_ref(a.paged ? a.paged + t : nullptr);
     p.T = a.T;
     p.n_empty = 0;
-    p.chunk_log2 = 3;  // kChunkBlocks
+    uint64_t total_blocks = 0;
+    for (int t = 0; t < a.T; ++t) total_blocks += cdiv(a.n[t], kBlock);
+    p.chunk_log2 = pick_chunk_log2(total_blocks, resident * NW);
     p.chunk_begin[0] = 0;
     for (int t = 0; t < a.T; ++t) {
         p.in[t] = static_cast<const uint8_t *>(a.in[t]);
@@ -829,7 +842,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
         p.n[t] = a.n[t];
         p.cap[t] = a.cap[t];
         const uint64_t nb = cdiv(a.n[t], kBlock);
-        p.chunk_begin[t + 1] = p.chunk_begin[t] + uint32_t(cdiv(nb, uint64_t(kChunkBlocks)));
+        p.chunk_begin[t + 1] = p.chunk_begin[t] + uint32_t(cdiv(nb, uint64_t(1) << p.chunk_log2));
         if (a.n[t] == 0) p.empty[p.n_empty++] = uint16_t(t);
     }
     p.total_chunks = p.chunk_begin[a.T];
@@ -837,6 +850,11 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     if (p.total_jobs == 0) return SZ_OK;
     const uint64_t need = cdiv(p.total_jobs, NW);
     const uint64_t grid = need < resident ? need : resident;
+    auto kern = kern_full;
+    if (p.chunk_log2 != kMaxChunkLog2) {
+        kern = kern_any;
+        if (resident_per_sm(reinterpret_cast<const void *>(kern_any), NT, smem, cache_any) < 1) return SZ_ERR_CUDA;
+    }
     kern<<<unsigned(grid), NT, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
