@@ -332,6 +332,39 @@ def run_ours(args, rank, world, device):
         st = sz.sz_last_device_status(w)
         if st != 0:
             raise RuntimeError("device status after timing: %s" % sz.sz_status_string(st))
+    if args.graph:
+        # The same step captured once as a CUDA graph and replayed: the calls
+        # launch kernels only (no allocation, no synchronisation), so they capture
+        # as they are; replay removes the host launch gaps between the calls.
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=device)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap), torch.cuda.graph(graph, stream=cap):
+            plan_all(); encode_all(); decode_all()
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(K):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        total_ms = g0.elapsed_time(g1)
+        for w in ws_g:
+            st = sz.sz_last_device_status(w)
+            if st != 0:
+                raise RuntimeError("device status after graph replay: %s" % sz.sz_status_string(st))
+        if not args.paged:
+            for x, d in zip(wl.xs, decs):
+                if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
+                    raise RuntimeError("round trip mismatch after graph replay")
+        del graph
 
     ms_step = max_over_ranks(total_ms / K, world, device)
     raw_all = sum_over_ranks(float(wl.raw_bytes), world, device)
@@ -363,6 +396,7 @@ def run_ours(args, rank, world, device):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "u8" if dt == 1 else "u16", "data": "synthetic (seeded generator, see DESIGN.md)",
         "config": {"workload": wl.name, "desc": wl.desc, "tensors_per_rank": T,
+                   "launch": "one CUDA graph per step" if args.graph else "direct launches",
                    "codebooks": "reused from a calibration plan (no histogram pass per step)" if args.reuse
                    else "own plan per step",
                    "layout": ("paged: %d-token pages, random page order in and out" % args.paged) if args.paged
@@ -609,6 +643,9 @@ def main():
                     help="hold the tensors in pages of TOKENS tokens (paged KV), in random page order")
     ap.add_argument("--transfer", action="store_true",
                     help="also run the layer-pipelined transfer (encode on the source, decode on the destination)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time the step with direct launches instead of one captured CUDA graph per step "
+                         "(per-kernel times always come from direct launches)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     args = ap.parse_args()
