@@ -47,6 +47,11 @@
  *     recorded in the workspace's device error word (the first error wins)
  *     and read, then cleared, by sz_last_device_status.  No call aborts,
  *     throws or traps the GPU.
+ *   - CUDA graphs: the plan, encode and decode calls (contiguous, paged, reuse)
+ *     only enqueue kernels on their stream -- no allocation, no synchronisation
+ *     -- so a sequence of them can be captured into a CUDA graph and replayed,
+ *     once each call has run on the device (its first call sets the kernel's
+ *     shared-memory limit).  The buffers captured are the ones replayed.
  *   - Workspaces: size with sz_workspace_bytes*, zero once with
  *     sz_workspace_init before first use.  The kernels leave it ready for the
  *     next call.  A workspace serves one stream at a time; calls that use the

@@ -193,3 +193,42 @@ def test_prepared_batch_matches_functional_calls():
             assert np.array_equal(dec.view(torch.uint8).cpu().numpy(), raw)
     with pytest.raises(ValueError):
         m.Batch(0, [torch.zeros(8, 8, dtype=torch.bfloat16, device="cuda").t()], [outs[0]], ws, plans)
+
+
+def test_calls_capture_into_a_cuda_graph():
+    """plan, encode and decode enqueue kernels only (no allocation, no
+    synchronisation), so a step captures into a CUDA graph; replays on new data in
+    the same buffers give the oracle's streams and exact round trips."""
+    m = sz()
+    rng = np.random.default_rng(41)
+    for dtype in (0, 1):
+        sizes = [4096 * 9 + 7, 70000, 0]
+        raws = [oracle_pins._kvlike(rng, n, dtype) for n in sizes]
+        xs = [from_raw(r, dtype) for r in raws]
+        ws = m.new_workspace(dtype, sizes)
+        plans = m.new_plans(len(xs))
+        outs = [torch.zeros(m.sz_max_compressed_size(dtype, n), dtype=torch.uint8, device="cuda") for n in sizes]
+        decs = [torch.empty_like(x) for x in xs]
+        b = m.Batch(dtype, xs, outs, ws, plans, decs=decs)
+        b.plan(); b.encode(); b.decode()            # first calls set each kernel up on the device
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s), torch.cuda.graph(graph, stream=s):
+            b.plan(); b.encode(); b.decode()
+        torch.cuda.current_stream().wait_stream(s)
+        for rep in range(2):
+            new = [oracle_pins._kvlike(rng, n, dtype) for n in sizes]
+            for x, r in zip(xs, new):
+                if r.size:
+                    x.view(torch.uint8).copy_(torch.from_numpy(r).cuda())
+            graph.replay()
+            torch.cuda.synchronize()
+            assert m.sz_last_device_status(ws) == 0
+            totals = m.sz_compressed_sizes(plans)
+            for r, out, tot, dec in zip(new, outs, totals, decs):
+                ref = oracle.encode(dtype, r)
+                assert tot == ref.size and np.array_equal(out[:tot].cpu().numpy(), ref)
+                assert np.array_equal(dec.view(torch.uint8).cpu().numpy(), r)
+        del graph
