@@ -11,17 +11,19 @@
 //     blocks and checks a tensor's header (and builds its code-pair table)
 //     when it moves to it; a stream that fails a check sets
 //     SZ_ERR_CORRUPT_STREAM and is not written;
-//   - the block's code and plane bytes (6 KB BF16, 3.5 KB E5M2) arrive by bulk
-//     copy into one of the warp's two shared-memory stages while the warp
-//     decodes the previous block (waits are bounded); the next block's
-//     offsets-table entries and first 32 escape bytes are prefetched into
-//     registers the same way;
-//   - per 256-element (BF16) or 512-element (E5M2) step: each code byte (two
-//     4-bit codes) selects a pre-spread exponent pair from a 256-entry shared
-//     table; escape ranks come from a warp prefix of per-lane counts and the
-//     escape bytes from a shuffle; the elements are reassembled with byte
-//     permutes and integer multiply-adds and written with 16-byte stores
-//     (512 contiguous bytes per warp instruction).
+//   - the block's code and plane bytes (6 KB BF16, 3.5 KB E5M2) arrive by 1-D
+//     bulk copies of 1.5-1.8 KB units into a 4-stage shared-memory ring that
+//     runs 2-3 units ahead of the decoding, across into the claimed next block
+//     (waits are bounded); the next block's offsets-table entries and first 32
+//     escape bytes are prefetched into registers;
+//   - per 256-element (BF16) or 512-element (E5M2) step: BF16 code bytes (two
+//     4-bit codes) select pre-spread exponent pairs from a 256-entry shared
+//     table, E5M2 codes select exponents from a 16-byte table in registers
+//     with prmt; escape ranks come from ballots (a fast path when no lane has
+//     two) and the escape bytes from a shuffle -- an E5M2 lane's single escape
+//     enters through its table's code-15 byte; the elements are reassembled
+//     with byte permutes and integer multiply-adds and written with 16-byte
+//     stores (512 contiguous bytes per warp instruction).
 #include <type_traits>
 
 #include "sz_common.cuh"
@@ -33,23 +35,36 @@ namespace {
 
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
-constexpr uint32_t kStageBytes = 1536;                // a quarter block's codes and planes (BF16 size)
-constexpr int kStages = 4;                            // ring of quarter-block stages per warp
+constexpr int kStages = 4;                            // ring of input-unit stages per warp
 constexpr uint64_t kWaitLimitNs = 1000000000ull;      // 1 s
 
-template <int DT>
+// Input units of the ring: quarter blocks for BF16 (1536 bytes of codes and
+// planes) and for paged E5M2 (whose pages are only known to hold multiples of
+// 1024 elements), half blocks for contiguous E5M2 (1792 bytes) -- so that a
+// unit is some 1.5-2 KB and its per-unit work covers several steps.
+template <int DT, bool PAGED = false>
 struct DGeo {
     static constexpr int LE = (DT == SZ_BF16) ? 8 : 16;   // elements per lane per step
     static constexpr int IT = int(kBlock) / (32 * LE);     // steps per block
-    static constexpr int QIT = IT / 4;                     // steps per quarter block
-    // quarter-block stage layout: codes, then plane a, then plane b
-    static constexpr uint32_t kCodeBytes = 512;
-    static constexpr uint32_t kABytes = (DT == SZ_BF16) ? 1024 : 128;
-    static constexpr uint32_t kBBytes = (DT == SZ_BF16) ? 0 : 256;
+    static constexpr int kUnits = (DT == SZ_BF16 || PAGED) ? 4 : 2;
+    static constexpr int QIT = IT / kUnits;                // steps per unit
+    static constexpr uint32_t kUnitElems = kBlock / kUnits;
+    // stage layout: codes, then plane a, then plane b
+    static constexpr uint32_t kCodeBytes = kUnitElems / 2;
+    static constexpr uint32_t kABytes = (DT == SZ_BF16) ? kUnitElems : kUnitElems / 8;
+    static constexpr uint32_t kBBytes = (DT == SZ_BF16) ? 0 : kUnitElems / 4;
     static constexpr uint32_t kA = kCodeBytes, kB = kCodeBytes + kABytes;
     static constexpr uint32_t kBytes = kCodeBytes + kABytes + kBBytes;
+    // units issued ahead of the one being decoded; the unit of a block at which
+    // the next block's claim must be known (its first unit gets issued there),
+    // and the one after, where the next block's first escapes are fetched
+    static constexpr int kAhead = kUnits == 4 ? 3 : 2;
+    static constexpr int kResolveQ = kUnits - kAhead;
+    static constexpr int kEscQ = kResolveQ + 1;
+    static_assert(kAhead < kStages && kEscQ < kUnits, "ring geometry");
 };
 
+template <uint32_t kStageBytes>
 struct alignas(128) WarpSmem {
     uint8_t stage[kStages][kStageBytes];
     uint32_t tab[256];       // code byte -> pre-spread exponent pair
@@ -72,23 +87,23 @@ struct WarpStream {
     uint32_t xt[4];               // E5M2: byte c = exponent of code c, times 4 (byte 15: 0)
 };
 
-// Step `it` (within a quarter block) from the shared-memory stage at address st.
-template <int DT>
+// Step `it` (within a unit) from the shared-memory stage at address st.
+template <int DT, typename G>
 __device__ __forceinline__ DFrag read_stage(uint32_t st, int it) {
     const uint32_t lane = threadIdx.x & 31;
     DFrag f;
     if constexpr (DT == SZ_BF16) {
         f.c0 = lds_u32(st + it * 128 + lane * 4);
         f.c1 = 0;
-        const uint2 s = lds_u64(st + DGeo<DT>::kA + it * 256 + lane * 8);
+        const uint2 s = lds_u64(st + G::kA + it * 256 + lane * 8);
         f.a = s.x;
         f.b = s.y;
     } else {
         const uint2 c = lds_u64(st + it * 256 + lane * 8);
         f.c0 = c.x;
         f.c1 = c.y;
-        f.a = lds_u16(st + DGeo<DT>::kA + it * 64 + lane * 2);
-        f.b = lds_u32(st + DGeo<DT>::kB + it * 128 + lane * 4);
+        f.a = lds_u16(st + G::kA + it * 64 + lane * 2);
+        f.b = lds_u32(st + G::kB + it * 128 + lane * 4);
     }
     return f;
 }
@@ -206,12 +221,10 @@ __device__ __forceinline__ StreamGeo stream_geo(const DecodeParams<MAXB> &p, int
     return g;
 }
 
-// Lane 0 starts the bulk copies of quarter q of block blk into a stage.
-template <int DT>
-__device__ __forceinline__ void issue_quarter(uint8_t *st, uint64_t *bar, const StreamGeo &sg,
-                                              uint64_t blk, int q) {
-    using G = DGeo<DT>;
-    const uint64_t u = blk * 4 + q;  // quarter index within the tensor
+// Lane 0 starts the bulk copies of unit q of block blk into a stage.
+template <typename G>
+__device__ __forceinline__ void issue_unit(uint8_t *st, uint64_t *bar, const StreamGeo &sg, uint64_t blk, int q) {
+    const uint64_t u = blk * G::kUnits + q;  // unit index within the tensor
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(bar, G::kBytes);
     bulk_g2s(st, sg.comp + sg.code + u * G::kCodeBytes, G::kCodeBytes, bar);
@@ -432,16 +445,16 @@ __device__ __forceinline__ uint32_t claim_resolve(const DecodeParams<MAXB> &p, i
     return 0;
 }
 
-// The warp's quarter-block units in claim order; the producer side of its
-// ring.  It runs three units ahead of the consumer, so it reaches the next
-// block's first quarter while the consumer is on the current block's second:
+// The warp's input units in claim order; the producer side of its ring.  It
+// runs G::kAhead units ahead of the consumer, so it reaches the next block's
+// first unit while the consumer is on unit G::kResolveQ of the current block:
 // the next block is handed over (set_next) just before that.
-template <int DT, int MAXB>
-struct QuarterFeed {
+template <int DT, int MAXB, typename G, typename WS>
+struct UnitFeed {
     static constexpr int kAwait = -2;
     int t;          // tensor of the next unit to issue; -1: no more units, kAwait: next block not yet known
     uint32_t blk;   // its block within the tensor
-    int q;          // its quarter
+    int q;          // its unit within the block
     bool full;      // the block has all 4096 elements (partial blocks are read directly)
     int sg_t;       // tensor whose geometry sg holds
     StreamGeo sg;
@@ -467,26 +480,27 @@ struct QuarterFeed {
     }
     // Issue the next unit into stage v % kStages (if it is part of a full
     // block); returns the bit to set in the issued mask.
-    __device__ __forceinline__ uint32_t issue_next(WarpSmem &W) {
+    __device__ __forceinline__ uint32_t issue_next(WS &W) {
         if (t < 0) return 0;
         const int st = int(v % kStages);
         uint32_t bit = 0;
         if (full) {
-            if ((threadIdx.x & 31) == 0) issue_quarter<DT>(W.stage[st], &W.bar[st], sg, blk, q);
+            if ((threadIdx.x & 31) == 0) issue_unit<G>(W.stage[st], &W.bar[st], sg, blk, q);
             bit = 1u << st;
         }
         ++v;
-        if (++q == 4) t = kAwait;
+        if (++q == G::kUnits) t = kAwait;
         return bit;
     }
 };
 
 template <int DT, int MAXB, bool PAGED>
 __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
-    using G = DGeo<DT>;
+    using G = DGeo<DT, PAGED>;
+    using WS = WarpSmem<G::kBytes>;
     extern __shared__ __align__(128) uint8_t s_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpSmem &W = reinterpret_cast<WarpSmem *>(s_raw)[warp];
+    WS &W = reinterpret_cast<WS *>(s_raw)[warp];
     const uint32_t tab_addr = smem_u32(W.tab);
     if (lane == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&W.bar[i], 1);
@@ -508,9 +522,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
     uint32_t issued = 0;  // bit s: stage s holds an issued unit not yet waited for
     uint32_t parity = 0;  // bit s: parity of stage s's next completion
     if (t >= 0) {
-        QuarterFeed<DT, MAXB> feed;
+        UnitFeed<DT, MAXB, G, WS> feed;
         feed.start(p, t, blk);
-        for (int k = 0; k < kStages - 1; ++k) issued |= feed.issue_next(W);
+        for (int k = 0; k < G::kAhead; ++k) issued |= feed.issue_next(W);
 
         WarpStream ws;
         warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
@@ -520,7 +534,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
 
         while (true) {
             const uint8_t *comp = p.comp[t];
-            uint32_t pend = 0;  // claim of the next block, resolved at the second quarter
+            uint32_t pend = 0;  // claim of the next block, resolved at unit G::kResolveQ
             if (lane == 0) pend = atomicAdd(p.claim + t * kClaimStride, 1u);
             int t_n = t;
             uint32_t blk_n = 0;
@@ -533,16 +547,16 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
             constexpr int EB = Dt<DT>::kElemBytes;
             uint8_t *out = p.out[t] + (uint64_t(blk) * kBlock + uint64_t(lane) * G::LE) * EB;
             const bool full = (uint64_t(blk) + 1) * kBlock <= ws.n;
-            // paged output: lane q < 4 looks up where quarter q of the block goes
+            // paged output: lane q < G::kUnits looks up where unit q of the block goes
             uint64_t qoff = 0;
             if constexpr (PAGED) {
-                if (lane < 4 && uint64_t(blk) * kBlock + uint64_t(lane) * (kBlock / 4) < ws.n)
-                    qoff = elem_offset<EB>(p.pg[t], uint64_t(blk) * kBlock + uint64_t(lane) * (kBlock / 4));
+                if (lane < G::kUnits && uint64_t(blk) * kBlock + uint64_t(lane) * G::kUnitElems < ws.n)
+                    qoff = elem_offset<EB>(p.pg[t], uint64_t(blk) * kBlock + uint64_t(lane) * G::kUnitElems);
             }
             uint32_t running = 0;
             bool bad = false, timed_out = false;
-            for (int q = 0; q < 4; ++q, ++v) {
-                if (q == 1) {
+            for (int q = 0; q < G::kUnits; ++q, ++v) {
+                if (q == G::kResolveQ) {
                     blk_n = claim_resolve<MAXB>(p, t_n, pend);
                     feed.set_next(p, t_n, blk_n);
                     if (t_n == t && ws.ok) be_n = load_offsets(comp, blk_n);
@@ -554,7 +568,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                     parity ^= 1u << st;
                     issued &= ~(1u << st);
                 }
-                if (q == 2 && t_n == t && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
+                if (q == G::kEscQ && t_n == t && ws.ok) esc_n = load_escape_reg(comp, ws, be_n);
                 if (ok && !timed_out) {
                     if (full) {
                         const uint32_t st_addr = smem_u32(W.stage[st]);
@@ -565,14 +579,14 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                             if (!store && lane == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
 #pragma unroll
                             for (int it = 0; it < G::QIT; ++it) {
-                                const DFrag f = read_stage<DT>(st_addr, it);
+                                const DFrag f = read_stage<DT, G>(st_addr, it);
                                 decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE, running,
                                                              esc_reg, esc_g, cnt, bad, store);
                             }
                         } else {
 #pragma unroll
                             for (int it = 0; it < G::QIT; ++it) {
-                                const DFrag f = read_stage<DT>(st_addr, it);
+                                const DFrag f = read_stage<DT, G>(st_addr, it);
                                 decode_step<DT, false>(f, tab_addr, ws.xt, out + (q * G::QIT + it) * 512, G::LE,
                                                        running, esc_reg, esc_g, cnt, bad);
                             }
@@ -654,7 +668,7 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel_paged(const __grid_consta
 template <int DT, int MAXB, bool PAGED>
 sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     auto kern = PAGED ? decode_kernel_paged<DT, MAXB> : decode_kernel<DT, MAXB>;
-    const size_t smem = sizeof(WarpSmem) * NW;
+    const size_t smem = sizeof(WarpSmem<DGeo<DT, PAGED>::kBytes>) * NW;
     static std::atomic<int> cache[kMaxDevices];
     const int per_sm = resident_per_sm(reinterpret_cast<const void *>(kern), NT, smem, cache);
     if (per_sm < 1) return SZ_ERR_CUDA;
