@@ -18,6 +18,7 @@ BF16 = 0
 E5M2 = 1
 
 OK, ERR_ARG, ERR_DTYPE, ERR_SMALL, ERR_CORRUPT = 0, 1, 2, 3, 4
+FLAG_RAW_BLOCKS = 1  # header byte 39, bit 0: blocks that would expand are stored raw
 
 _u8p = ctypes.POINTER(ctypes.c_uint8)
 _u64p = ctypes.POINTER(ctypes.c_uint64)
@@ -55,6 +56,9 @@ class Oracle:
         L.orc_encode.restype = ctypes.c_int64
         L.orc_encode_codebook.argtypes = [ctypes.c_int, _u8p, ctypes.c_uint64, _u8p, _u8p, ctypes.c_uint64]
         L.orc_encode_codebook.restype = ctypes.c_int64
+        L.orc_encode_ex.argtypes = [ctypes.c_int, _u8p, ctypes.c_uint64, _u8p, ctypes.c_uint,
+                                    _u8p, ctypes.c_uint64]
+        L.orc_encode_ex.restype = ctypes.c_int64
         L.orc_decode.argtypes = [_u8p, ctypes.c_uint64, _u8p, ctypes.c_uint64]
         L.orc_decode.restype = ctypes.c_int
         self.lib = L
@@ -82,26 +86,54 @@ class Oracle:
             raise ValueError("orc_codebook failed: %d" % rc)
         return cb
 
-    def encode_status(self, dtype: int, x, cap=None):
-        """Encode; return (bytes written or -error, stream as uint8)."""
+    def encode_ex_status(self, dtype: int, x, cb=None, raw_blocks=False, cap=None):
+        """Encode with the tensor's own codebook (cb None) or a given one, with or
+        without raw blocks; return (bytes written or -error, stream as uint8)."""
         raw = _raw(x)
         n = raw.size // elem_size(dtype)
+        cbp = None
+        if cb is not None:
+            cbv = np.ascontiguousarray(np.asarray(cb, dtype=np.uint8).reshape(-1))
+            if cbv.size != 15:
+                raise ValueError("a codebook has 15 entries")
+            cbp = _u8(cbv)
         if cap is None:
             cap = self.compressed_size(dtype, n, n)
         # poisoned, so that a stream byte the encoder forgets to write shows up
         out = np.full(max(cap, 1), 0xA5, dtype=np.uint8)
+        flags = FLAG_RAW_BLOCKS if raw_blocks else 0
+        r = int(self.lib.orc_encode_ex(dtype, _u8(raw), n, cbp, flags, _u8(out), cap))
+        return r, (out[:r].copy() if r >= 0 else out[:0])
+
+    def encode_ex(self, dtype: int, x, cb=None, raw_blocks=False) -> np.ndarray:
+        r, out = self.encode_ex_status(dtype, x, cb, raw_blocks)
+        if r < 0:
+            raise ValueError("orc_encode_ex failed: %d" % -r)
+        return out
+
+    def encode_status(self, dtype: int, x, cap=None, raw_blocks=False):
+        """Encode; return (bytes written or -error, stream as uint8)."""
+        if raw_blocks:
+            return self.encode_ex_status(dtype, x, None, True, cap)
+        raw = _raw(x)
+        n = raw.size // elem_size(dtype)
+        if cap is None:
+            cap = self.compressed_size(dtype, n, n)
+        out = np.full(max(cap, 1), 0xA5, dtype=np.uint8)
         r = int(self.lib.orc_encode(dtype, _u8(raw), n, _u8(out), cap))
         return r, (out[:r].copy() if r >= 0 else out[:0])
 
-    def encode(self, dtype: int, x) -> np.ndarray:
+    def encode(self, dtype: int, x, raw_blocks=False) -> np.ndarray:
         """Encode raw elements (numpy array or bytes); return the stream as uint8."""
-        r, out = self.encode_status(dtype, x)
+        r, out = self.encode_status(dtype, x, raw_blocks=raw_blocks)
         if r < 0:
             raise ValueError("orc_encode failed: %d" % -r)
         return out
 
-    def encode_codebook_status(self, dtype: int, x, cb, cap=None):
+    def encode_codebook_status(self, dtype: int, x, cb, cap=None, raw_blocks=False):
         """Encode with the given 15-entry codebook; return (bytes written or -error, stream)."""
+        if raw_blocks:
+            return self.encode_ex_status(dtype, x, cb, True, cap)
         raw = _raw(x)
         n = raw.size // elem_size(dtype)
         cbv = np.ascontiguousarray(np.asarray(cb, dtype=np.uint8).reshape(-1))
@@ -113,9 +145,9 @@ class Oracle:
         r = int(self.lib.orc_encode_codebook(dtype, _u8(raw), n, _u8(cbv), _u8(out), cap))
         return r, (out[:r].copy() if r >= 0 else out[:0])
 
-    def encode_codebook(self, dtype: int, x, cb) -> np.ndarray:
+    def encode_codebook(self, dtype: int, x, cb, raw_blocks=False) -> np.ndarray:
         """Encode raw elements with a given codebook (codebook reuse); return the stream."""
-        r, out = self.encode_codebook_status(dtype, x, cb)
+        r, out = self.encode_codebook_status(dtype, x, cb, raw_blocks=raw_blocks)
         if r < 0:
             raise ValueError("orc_encode_codebook failed: %d" % -r)
         return out
@@ -157,20 +189,20 @@ def codebook(dtype, hist):
     return default().codebook(dtype, hist)
 
 
-def encode(dtype, x):
-    return default().encode(dtype, x)
+def encode(dtype, x, raw_blocks=False):
+    return default().encode(dtype, x, raw_blocks)
 
 
-def encode_status(dtype, x, cap=None):
-    return default().encode_status(dtype, x, cap)
+def encode_status(dtype, x, cap=None, raw_blocks=False):
+    return default().encode_status(dtype, x, cap, raw_blocks)
 
 
-def encode_codebook(dtype, x, cb):
-    return default().encode_codebook(dtype, x, cb)
+def encode_codebook(dtype, x, cb, raw_blocks=False):
+    return default().encode_codebook(dtype, x, cb, raw_blocks)
 
 
-def encode_codebook_status(dtype, x, cb, cap=None):
-    return default().encode_codebook_status(dtype, x, cb, cap)
+def encode_codebook_status(dtype, x, cb, cap=None, raw_blocks=False):
+    return default().encode_codebook_status(dtype, x, cb, cap, raw_blocks)
 
 
 def decode(stream, n, dtype):

@@ -36,6 +36,20 @@
  *           byte i/4), code plane, escapes
  *   All padding bytes and unused high bits are zero.
  *
+ * Header byte 39 holds flags; bit 0 allows raw blocks.  Without it every
+ * block is coded as above.  With it, a block of m elements whose escapes
+ * would fill at least K = ceil(m/2) bytes (BF16) or ceil(m/8) bytes (E5M2) --
+ * the size of its exponent bits above the low four -- is stored raw: its code
+ * nibbles hold the low four bits of each exponent and its K escape-section
+ * bytes the remaining bits (BF16: the high nibble of element j's exponent in
+ * nibble j%2 of byte j/2; E5M2: bit 4 of element j's exponent at bit j%8 of
+ * byte j/8; j counted within the block).  The offsets table counts K bytes
+ * for such a block, and a coded block always has fewer than K escapes, so a
+ * decoder tells the two apart by the count.  E in the header is the length
+ * of the escape section.  A raw block costs exactly its raw bytes, so no
+ * block expands.  The pages describe no such fallback; it is this format's
+ * own extension for data whose exponents the codebook does not capture.
+ *
  * Every loop below walks the elements one at a time, in order.  No blocking,
  * no vector tricks: a reader can check each step against the description.
  */
@@ -60,6 +74,7 @@ enum {
 #define ORC_BLOCK 4096u
 #define ORC_CODES 15u          /* codes 0..14 name codebook entries          */
 #define ORC_ESCAPE 15u         /* code 15 marks an escaped exponent          */
+#define ORC_FLAG_RAW_BLOCKS 1u /* header byte 39, bit 0: raw blocks allowed  */
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -206,33 +221,78 @@ static unsigned code_of(const uint8_t *cb, unsigned e)
     return ORC_ESCAPE;
 }
 
-/* Encode n elements into out (capacity cap bytes) with the codebook cb[15]
- * given by the caller instead of the tensor's own.  Any 15 distinct exponent
+/* Elements of block b of a tensor of n elements. */
+static uint64_t block_elems(uint64_t n, uint64_t b)
+{
+    uint64_t first = b * ORC_BLOCK;
+    return n - first < ORC_BLOCK ? n - first : ORC_BLOCK;
+}
+
+/* Escape-section bytes of a raw block of m elements: its exponent bits above
+ * the low four (four per BF16 element, one per E5M2 element). */
+static uint64_t raw_block_bytes(int dtype, uint64_t m)
+{
+    return dtype == ORC_BF16 ? ceil_div(m, 2) : ceil_div(m, 8);
+}
+
+/* Whether block b is stored raw: raw blocks are allowed and the block's
+ * escapes under cb would fill at least raw_block_bytes. */
+static int block_is_raw(int dtype, const uint8_t *in, uint64_t n, const uint8_t *cb, unsigned flags,
+                        uint64_t b)
+{
+    if (!(flags & ORC_FLAG_RAW_BLOCKS)) return 0;
+    uint64_t m = block_elems(n, b), escapes = 0;
+    for (uint64_t i = b * ORC_BLOCK; i < b * ORC_BLOCK + m; i++)
+        if (code_of(cb, exponent_of(dtype, element_bits(dtype, in, i))) == ORC_ESCAPE) escapes++;
+    return escapes >= raw_block_bytes(dtype, m);
+}
+
+/* Encode n elements into out (capacity cap bytes).  cb_given: a codebook of
+ * 15 exponent values chosen by the caller, or NULL for the tensor's own (its
+ * 15 most frequent exponent values, Abstract).  Any 15 distinct exponent
  * values of the dtype's range form a valid codebook, and the result is still
  * lossless: exponents outside it take the escape path (SplitZip project page,
  * Abstract: rare exponent values go through the sparse escape stream).  This
  * is what lets a codebook found once be reused for other layers or later
  * steps without a new histogram pass (the related-work list of the ZipServ
  * page names exponent reuse across iterations: "CIERA: Cross-Iteration
- * Exponent Reuse for Lossless Allgather in Sharded MoE Training").  The
- * stream is an ordinary format-v1 stream: its header records cb and the
- * escape count E that cb leaves.
+ * Exponent Reuse for Lossless Allgather in Sharded MoE Training").
+ * flags: 0, or ORC_FLAG_RAW_BLOCKS to let blocks that would expand be stored
+ * raw (see the format above).
  * Returns the stream length, or minus an ORC_ERR_* code. */
-int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint8_t *cb,
-                            uint8_t *out, uint64_t cap)
+int64_t orc_encode_ex(int dtype, const uint8_t *in, uint64_t n, const uint8_t *cb_given, unsigned flags,
+                      uint8_t *out, uint64_t cap)
 {
     if (dtype != ORC_BF16 && dtype != ORC_E5M2) return -ORC_ERR_DTYPE;
-    if ((n && !in) || !out || !cb || n >= (1ull << 32)) return -ORC_ERR_ARG;
-    for (unsigned c = 0; c < ORC_CODES; c++) {
-        if (cb[c] >= exponent_values(dtype)) return -ORC_ERR_ARG;
-        for (unsigned d = 0; d < c; d++)
-            if (cb[d] == cb[c]) return -ORC_ERR_ARG;
+    if ((n && !in) || !out || n >= (1ull << 32)) return -ORC_ERR_ARG;
+    if (flags & ~ORC_FLAG_RAW_BLOCKS) return -ORC_ERR_ARG;
+    uint8_t own[ORC_CODES];
+    const uint8_t *cb = cb_given;
+    if (cb) {
+        for (unsigned c = 0; c < ORC_CODES; c++) {
+            if (cb[c] >= exponent_values(dtype)) return -ORC_ERR_ARG;
+            for (unsigned d = 0; d < c; d++)
+                if (cb[d] == cb[c]) return -ORC_ERR_ARG;
+        }
+    } else {
+        uint64_t hist[256];
+        orc_histogram(dtype, in, n, hist);
+        orc_codebook(dtype, hist, own);
+        cb = own;
     }
 
-    /* 1. escape count: every element whose exponent is not in the codebook */
+    /* 1. escape count: every element whose exponent is not in the codebook
+     *    (a raw block instead counts its raw_block_bytes) */
     uint64_t E = 0;
-    for (uint64_t i = 0; i < n; i++)
-        if (code_of(cb, exponent_of(dtype, element_bits(dtype, in, i))) == ORC_ESCAPE) E++;
+    uint64_t nb = ceil_div(n, ORC_BLOCK);
+    for (uint64_t b = 0; b < nb; b++) {
+        if (block_is_raw(dtype, in, n, cb, flags, b)) {
+            E += raw_block_bytes(dtype, block_elems(n, b));
+            continue;
+        }
+        for (uint64_t i = b * ORC_BLOCK; i < b * ORC_BLOCK + block_elems(n, b); i++)
+            if (code_of(cb, exponent_of(dtype, element_bits(dtype, in, i))) == ORC_ESCAPE) E++;
+    }
 
     orc_layout L = layout_of(dtype, n, E);
     if (cap < L.total) return -ORC_ERR_SMALL;
@@ -246,17 +306,24 @@ int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint
     put_u64(out + 8, n);
     put_u64(out + 16, E);
     for (unsigned c = 0; c < ORC_CODES; c++) out[24 + c] = cb[c];
-    out[39] = 0;
+    out[39] = (uint8_t)flags;
     put_u64(out + 40, L.total);
 
     /* 3. one pass in element order: planes, codes, escapes, and the escape
      *    count before each block (the exclusive prefix over blocks). */
-    uint64_t k = 0;  /* escapes emitted so far */
+    uint64_t k = 0;      /* escape-section bytes emitted so far */
+    int raw = 0;         /* the current block is stored raw      */
+    uint64_t k_raw = 0;  /* where a raw block's high bits start  */
     for (uint64_t i = 0; i < n; i++) {
         if (i % ORC_BLOCK == 0) put_u32(out + 64 + 4 * (i / ORC_BLOCK), (uint32_t)k);
+        if (i % ORC_BLOCK == 0) {
+            raw = block_is_raw(dtype, in, n, cb, flags, i / ORC_BLOCK);
+            k_raw = k;
+            if (raw) k += raw_block_bytes(dtype, block_elems(n, i / ORC_BLOCK));
+        }
         unsigned bits = element_bits(dtype, in, i);
         unsigned s = sign_of(dtype, bits), e = exponent_of(dtype, bits), m = mantissa_of(dtype, bits);
-        unsigned c = code_of(cb, e);
+        unsigned c = raw ? (e & 0xFu) : code_of(cb, e);
         if (dtype == ORC_BF16) {
             out[L.sec[0] + i] = (uint8_t)((s << 7) | m);
         } else {
@@ -265,7 +332,13 @@ int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint
         }
         uint64_t code_plane = L.sec[L.nsec - 1];
         out[code_plane + i / 2] |= (uint8_t)(c << (4 * (i % 2)));
-        if (c == ORC_ESCAPE) {
+        if (raw) {
+            uint64_t j = i % ORC_BLOCK;  /* position within the block */
+            if (dtype == ORC_BF16)
+                out[L.esc + k_raw + j / 2] |= (uint8_t)((e >> 4) << (4 * (j % 2)));
+            else
+                out[L.esc + k_raw + j / 8] |= (uint8_t)((e >> 4) << (j % 8));
+        } else if (c == ORC_ESCAPE) {
             out[L.esc + k] = (uint8_t)e;
             k++;
         }
@@ -274,25 +347,28 @@ int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint
     return (int64_t)L.total;
 }
 
+/* Encode with a codebook given by the caller (codebook reuse), no raw blocks.
+ * Returns the stream length, or minus an ORC_ERR_* code. */
+int64_t orc_encode_codebook(int dtype, const uint8_t *in, uint64_t n, const uint8_t *cb,
+                            uint8_t *out, uint64_t cap)
+{
+    if (!cb) return -ORC_ERR_ARG;
+    return orc_encode_ex(dtype, in, n, cb, 0u, out, cap);
+}
+
 /* Encode n elements into out (capacity cap bytes) with the tensor's own
- * codebook: its 15 most frequent exponent values (Abstract).
+ * codebook: its 15 most frequent exponent values (Abstract), no raw blocks.
  * Returns the stream length, or minus an ORC_ERR_* code. */
 int64_t orc_encode(int dtype, const uint8_t *in, uint64_t n, uint8_t *out, uint64_t cap)
 {
-    if (dtype != ORC_BF16 && dtype != ORC_E5M2) return -ORC_ERR_DTYPE;
-    if ((n && !in) || !out || n >= (1ull << 32)) return -ORC_ERR_ARG;
-    uint64_t hist[256];
-    uint8_t cb[ORC_CODES];
-    orc_histogram(dtype, in, n, hist);
-    orc_codebook(dtype, hist, cb);
-    return orc_encode_codebook(dtype, in, n, cb, out, cap);
+    return orc_encode_ex(dtype, in, n, NULL, 0u, out, cap);
 }
 
 /* Read and check a stream header.  On success fills dtype, n, E, cb and the
  * layout.  Checks are the ones a decoder needs to stay inside the buffer and
  * to reject streams this format cannot produce. */
 static int parse_header(const uint8_t *comp, uint64_t comp_bytes, int *dtype, uint64_t *n,
-                        uint64_t *E, uint8_t *cb, orc_layout *L)
+                        uint64_t *E, uint8_t *cb, unsigned *flags, orc_layout *L)
 {
     if (!comp || comp_bytes < 64) return ORC_ERR_CORRUPT;
     if (get_u32(comp) != ORC_MAGIC) return ORC_ERR_CORRUPT;
@@ -310,6 +386,8 @@ static int parse_header(const uint8_t *comp, uint64_t comp_bytes, int *dtype, ui
         for (unsigned d = 0; d < c; d++)
             if (cb[d] == cb[c]) return ORC_ERR_CORRUPT;
     }
+    *flags = comp[39];
+    if (*flags & ~ORC_FLAG_RAW_BLOCKS) return ORC_ERR_CORRUPT;
     *L = layout_of(*dtype, *n, *E);
     if (get_u64(comp + 40) != L->total) return ORC_ERR_CORRUPT;
     if (comp_bytes < L->total) return ORC_ERR_CORRUPT;
@@ -323,20 +401,40 @@ int orc_decode(const uint8_t *comp, uint64_t comp_bytes, uint8_t *out, uint64_t 
     int dtype;
     uint64_t sn, E;
     uint8_t cb[ORC_CODES];
+    unsigned flags;
     orc_layout L;
-    int rc = parse_header(comp, comp_bytes, &dtype, &sn, &E, cb, &L);
+    int rc = parse_header(comp, comp_bytes, &dtype, &sn, &E, cb, &flags, &L);
     if (rc) return rc;
     if (sn != n) return ORC_ERR_ARG;
     if (n && !out) return ORC_ERR_ARG;
 
-    uint64_t k = 0;  /* escapes consumed so far */
+    uint64_t k = 0;      /* escape-section bytes consumed so far */
+    int raw = 0;         /* the current block is stored raw       */
+    uint64_t k_raw = 0;  /* where a raw block's high bits start   */
     for (uint64_t i = 0; i < n; i++) {
         if (i % ORC_BLOCK == 0 && get_u32(comp + 64 + 4 * (i / ORC_BLOCK)) != k)
             return ORC_ERR_CORRUPT;  /* stored block offset disagrees */
+        if (i % ORC_BLOCK == 0) {
+            /* a block is raw exactly when its count is raw_block_bytes: a
+             * coded block has fewer escapes than that */
+            uint64_t next = get_u32(comp + 64 + 4 * (i / ORC_BLOCK + 1));
+            uint64_t K = raw_block_bytes(dtype, block_elems(n, i / ORC_BLOCK));
+            raw = (flags & ORC_FLAG_RAW_BLOCKS) && next >= k && next - k == K;
+            k_raw = k;
+            if (raw) {
+                if (next > E) return ORC_ERR_CORRUPT;
+                k = next;
+            }
+        }
         uint64_t code_plane = L.sec[L.nsec - 1];
         unsigned c = (comp[code_plane + i / 2] >> (4 * (i % 2))) & 0xFu;
         unsigned e;
-        if (c < ORC_CODES) {
+        if (raw) {
+            uint64_t j = i % ORC_BLOCK;  /* position within the block */
+            unsigned high = dtype == ORC_BF16 ? (comp[L.esc + k_raw + j / 2] >> (4 * (j % 2))) & 0xFu
+                                              : (comp[L.esc + k_raw + j / 8] >> (j % 8)) & 1u;
+            e = (high << 4) | c;
+        } else if (c < ORC_CODES) {
             e = cb[c];
         } else {
             if (k >= E) return ORC_ERR_CORRUPT;  /* more escapes than the header says */

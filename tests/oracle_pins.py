@@ -21,6 +21,12 @@ what:
                   is the tensor's own (found by numpy), the reader-checked v1
                   encoding under any other, a hand-worked golden stream
                   (bf16_n17_reuse.txt), and refusal of invalid codebooks
+  raw blocks      with header flag bit 0: hand-worked golden streams
+                  (bf16_n17_raw.txt, e5m2_n17_raw.txt), the exact threshold
+                  (K - 1 escapes coded, K raw), the ordinary stream when no
+                  block reaches it, no block above its raw bytes (closed form
+                  for uniform random bits), mixed streams checked by the
+                  independent reader, every bit pattern round-trips
 """
 import itertools
 import os
@@ -38,7 +44,7 @@ GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 def load_golden(path):
     """Parse a golden fixture: returns (dtype, raw input bytes, expected stream).
     A fixture with a `codebook` line was encoded with that given codebook; see
-    golden_codebook()."""
+    golden_codebook().  A `flags 1` line means raw blocks were allowed."""
     dtype = n = total = None
     raw = None
     at = []
@@ -57,7 +63,7 @@ def load_golden(path):
             elif key == "input_hex":
                 words = [int(w, 16) for w in rest.split()]
                 raw = np.array(words, dtype="<u2" if dtype == 0 else np.uint8).view(np.uint8)
-            elif key == "codebook":
+            elif key in ("codebook", "flags"):
                 pass
             elif key == "at":
                 off, _, hexes = rest.partition(":")
@@ -81,6 +87,16 @@ def golden_codebook(path):
     return None
 
 
+def golden_flags(path):
+    """The header flags a fixture was encoded with (0 unless a `flags` line says)."""
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line.startswith("flags "):
+                return int(line.split()[1])
+    return 0
+
+
 def golden_files():
     return sorted(os.path.join(GOLDEN_DIR, f) for f in os.listdir(GOLDEN_DIR) if f.endswith(".txt")
                   and f != "README.txt")
@@ -90,7 +106,8 @@ def pin_golden(orc):
     for path in golden_files():
         dtype, raw, expect = load_golden(path)
         cb = golden_codebook(path)
-        got = orc.encode(dtype, raw) if cb is None else orc.encode_codebook(dtype, raw, cb)
+        rb = golden_flags(path) == 1
+        got = orc.encode(dtype, raw, raw_blocks=rb) if cb is None else orc.encode_codebook(dtype, raw, cb, raw_blocks=rb)
         assert got.size == expect.size, (path, got.size, expect.size)
         diff = np.nonzero(got != expect)[0]
         assert diff.size == 0, (path, "first differing byte", int(diff[0]))
@@ -303,5 +320,110 @@ def pin_codebook_reuse(orc):
             assert orc.encode_codebook_status(dtype, raw, big)[0] == -oracle.ERR_ARG
 
 
+# -------------------------------------------------------------- raw blocks
+
+def _threshold_block(rng, dtype, escapes):
+    """One full 4096-element block whose own codebook leaves exactly `escapes`
+    escapes: 15 frequent exponents share the rest, and the escaped elements are
+    spread over rare exponents that each occur less often than any frequent one."""
+    common = np.arange(100, 115) if dtype == 0 else np.arange(8, 23)
+    rare = (np.arange(20, 84) if dtype == 0 else np.concatenate([np.arange(0, 8), np.arange(23, 32)]))
+    n_common = BLOCK_ELEMS - escapes
+    e = np.concatenate([np.resize(common, n_common), np.resize(rare, escapes)])
+    rng.shuffle(e)
+    if dtype == 0:
+        return ((rng.integers(0, 2, e.size) << 15) | (e << 7) | rng.integers(0, 128, e.size)).astype("<u2").view(np.uint8)
+    return ((rng.integers(0, 2, e.size) << 7) | (e << 2) | rng.integers(0, 4, e.size)).astype(np.uint8)
+
+
+BLOCK_ELEMS = 4096
+
+
+def pin_raw_blocks(orc):
+    """Raw blocks (header flag bit 0): checked field by field by the independent
+    reader; the threshold is exact (K - 1 escapes stay coded, K go raw); data
+    whose blocks never reach it gives the ordinary stream with only the flag
+    byte changed; no block ever expands, so a stream is at most the raw bytes
+    plus header, table and section padding; lossless on every bit pattern."""
+    rng = np.random.default_rng(99)
+    for dtype in (0, 1):
+        es = 2 if dtype == 0 else 1
+        K = 2048 if dtype == 0 else 512
+        # the threshold, in a block of its own and next to other blocks
+        for escapes, is_raw in ((K - 1, False), (K, True), (K + 1, True)):
+            blk = _threshold_block(rng, dtype, escapes)
+            st = orc.encode(dtype, blk, raw_blocks=True)
+            fieldcodec.check(st, blk, dtype, raw_blocks=True)
+            f = fieldcodec.parse(st)
+            assert f["E"] == (K if is_raw else escapes), (dtype, escapes, f["E"])
+            plain = orc.encode(dtype, blk)
+            if not is_raw:
+                same = plain.copy()
+                same[39] = 1
+                assert np.array_equal(st, same)
+            else:
+                assert st.size == plain.size - (escapes - K)
+            assert np.array_equal(orc.decode(st, BLOCK_ELEMS, dtype), blk)
+        # KV-like data: no block reaches the threshold; only the flag differs
+        for n in (1, 4095, 4097, 20000):
+            raw = _kvlike(rng, n, dtype)
+            st = orc.encode(dtype, raw, raw_blocks=True)
+            same = orc.encode(dtype, raw)
+            same[39] = 1
+            assert np.array_equal(st, same)
+        # uniform random bits: every block raw; closed-form size; never above raw
+        for n in RAGGED_N:
+            raw = rng.integers(0, 256, n * es).astype(np.uint8)
+            st = orc.encode(dtype, raw, raw_blocks=True)
+            fieldcodec.check(st, raw, dtype, raw_blocks=True)
+            sizes = fieldcodec.block_sizes(n)
+            escaped = fieldcodec.parse(orc.encode(dtype, raw))["offsets"]
+            all_raw = all(int(escaped[b + 1] - escaped[b]) >= fieldcodec.raw_block_bytes(dtype, m)
+                          for b, m in enumerate(sizes))
+            E_raw = sum(fieldcodec.raw_block_bytes(dtype, m) for m in sizes)
+            if all_raw:
+                assert fieldcodec.parse(st)["E"] == E_raw
+            layout = fieldcodec.layout(dtype, n, fieldcodec.parse(st)["E"])
+            assert st.size == layout[4]
+            table = fieldcodec.align256(64 + 4 * (layout[0] + 1))
+            assert st.size <= table + raw.size + 256 * len(layout[2]), (dtype, n, st.size)
+            assert np.array_equal(orc.decode(st, n, dtype), raw)
+        # blocks of both kinds in one stream, partial last block included
+        parts = [_kvlike(rng, 4096, dtype), rng.integers(0, 256, 4096 * es).astype(np.uint8),
+                 _kvlike(rng, 4096, dtype), rng.integers(0, 256, 1500 * es).astype(np.uint8)]
+        raw = np.concatenate(parts)
+        n = raw.size // es
+        st = orc.encode(dtype, raw, raw_blocks=True)
+        fieldcodec.check(st, raw, dtype, raw_blocks=True)
+        counts = np.diff(fieldcodec.parse(st)["offsets"])
+        assert counts[1] == K and counts[3] == fieldcodec.raw_block_bytes(dtype, 1500)
+        assert counts[0] < K and counts[2] < K
+        assert np.array_equal(orc.decode(st, n, dtype), raw)
+        # a codebook that holds nothing of the data: every block raw, still lossless
+        raw = _kvlike(rng, 9000, dtype)
+        e = set(fieldcodec.exponents(raw, dtype).tolist())
+        nbins = 256 if dtype == 0 else 32
+        absent = [v for v in range(nbins) if v not in e]
+        if len(absent) >= 15:
+            cb = np.array(absent[:15], dtype=np.uint8)
+            st = orc.encode_codebook(dtype, raw, cb, raw_blocks=True)
+            fieldcodec.check(st, raw, dtype, codebook=cb, raw_blocks=True)
+            assert fieldcodec.parse(st)["E"] == sum(fieldcodec.raw_block_bytes(dtype, m)
+                                                   for m in fieldcodec.block_sizes(9000))
+            assert np.array_equal(orc.decode(st, 9000, dtype), raw)
+    # every bit pattern, with raw blocks allowed
+    allp = np.arange(65536, dtype=np.uint32).astype("<u2")
+    shuffled = allp[np.random.default_rng(0).permutation(allp.size)]
+    for x in (allp, shuffled):
+        st = orc.encode(0, x.view(np.uint8), raw_blocks=True)
+        fieldcodec.check(st, x.view(np.uint8), 0, raw_blocks=True)
+        assert np.array_equal(orc.decode(st, 65536, 0), x.view(np.uint8))
+    e5 = np.repeat(np.arange(256, dtype=np.uint8), 33)
+    st = orc.encode(1, e5, raw_blocks=True)
+    fieldcodec.check(st, e5, 1, raw_blocks=True)
+    assert np.array_equal(orc.decode(st, e5.size, 1), e5)
+
+
 ALL_PINS = (pin_golden, pin_exhaustive_bf16, pin_exhaustive_e5m2, pin_ragged_sizes,
-            pin_bruteforce_codebook, pin_special_cases, pin_ratio_ceiling, pin_codebook_reuse)
+            pin_bruteforce_codebook, pin_special_cases, pin_ratio_ceiling, pin_codebook_reuse,
+            pin_raw_blocks)

@@ -37,7 +37,7 @@ CORRUPTIONS = {
     "E_too_large": lambda s, f: s.__setitem__(slice(16, 24), np.frombuffer(np.uint64(f["n"] + 1).tobytes(), np.uint8)),
     "total_wrong": lambda s, f: s.__setitem__(40, s[40] ^ 1),
     "cb_duplicate": lambda s, f: s.__setitem__(25, s[24]),
-    "cb_pad_nonzero": lambda s, f: s.__setitem__(39, 1),
+    "unknown_flag": lambda s, f: s.__setitem__(39, 2),
     "offset_tampered": lambda s, f: s.__setitem__(64 + 4, s[64 + 4] ^ 1),
     "first_offset": lambda s, f: s.__setitem__(64, 1),
     "last_offset": lambda s, f: s.__setitem__(64 + 4 * f["nb"], s[64 + 4 * f["nb"]] ^ 1),

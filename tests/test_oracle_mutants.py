@@ -50,9 +50,22 @@ MUTANTS = {
     "table_one_entry_short": [("64u + 4u * (L.nb + 1u)", "64u + 4u * L.nb", 1)],
     "given_codebook_duplicates_accepted": [("if (cb[d] == cb[c]) return -ORC_ERR_ARG;", "(void)d;", 1)],
     "given_codebook_replaced_by_own": [
-        ("    /* 1. escape count: every element whose exponent is not in the codebook */",
-         "    uint64_t own_h[256];\n    uint8_t own_cb[ORC_CODES];\n"
-         "    orc_histogram(dtype, in, n, own_h);\n    orc_codebook(dtype, own_h, own_cb);\n    cb = own_cb;", 1)],
+        ("    uint64_t E = 0;\n    uint64_t nb = ceil_div(n, ORC_BLOCK);",
+         "    uint64_t own_h[256];\n    uint8_t own_cb2[ORC_CODES];\n"
+         "    orc_histogram(dtype, in, n, own_h);\n    orc_codebook(dtype, own_h, own_cb2);\n    cb = own_cb2;\n"
+         "    uint64_t E = 0;\n    uint64_t nb = ceil_div(n, ORC_BLOCK);", 1)],
+    # raw blocks
+    "raw_threshold_strict": [("return escapes >= raw_block_bytes(dtype, m);",
+                              "return escapes > raw_block_bytes(dtype, m);", 1)],
+    "raw_blocks_never_taken": [("    if (!(flags & ORC_FLAG_RAW_BLOCKS)) return 0;\n", "    return 0;\n", 1)],
+    "raw_flag_not_written": [("out[39] = (uint8_t)flags;", "out[39] = 0;", 1)],
+    "raw_high_nibbles_swapped": [("(4 * (j % 2))", "(4 * (1 - j % 2))", None)],
+    "raw_e5m2_bitmap_msb_first": [("(j % 8)", "(7 - j % 8)", None)],
+    "raw_low_bits_shifted": [("unsigned c = raw ? (e & 0xFu) : code_of(cb, e);",
+                              "unsigned c = raw ? ((e >> 1) & 0xFu) : code_of(cb, e);", 1),
+                             ("e = (high << 4) | c;", "e = (high << 4) | (c << 1);", 1)],
+    "raw_block_bytes_bf16_quarter": [("return dtype == ORC_BF16 ? ceil_div(m, 2) : ceil_div(m, 8);",
+                                      "return dtype == ORC_BF16 ? ceil_div(m, 4) : ceil_div(m, 8);", 1)],
 }
 
 

@@ -19,6 +19,7 @@ def test_exhaustive_bf16_odd_repeats(orc):
 def test_golden_fixtures_present():
     names = [f.rsplit("/", 1)[-1] for f in oracle_pins.golden_files()]
     assert "bf16_n17.txt" in names and "e5m2_n17.txt" in names
+    assert "bf16_n17_raw.txt" in names and "e5m2_n17_raw.txt" in names
 
 
 def test_encode_reports_small_buffer(orc):
@@ -56,6 +57,7 @@ CORRUPTIONS = {
     "E_too_large": lambda s, f: s.__setitem__(slice(16, 24), np.frombuffer(np.uint64(f["n"] + 1).tobytes(), np.uint8)),
     "total_wrong": lambda s, f: s.__setitem__(40, s[40] ^ 1),
     "cb_duplicate": lambda s, f: s.__setitem__(25, s[24]),
+    "unknown_flag": lambda s, f: s.__setitem__(39, 2),
     "offset_tampered": lambda s, f: s.__setitem__(64 + 4, s[64 + 4] ^ 1),
     "last_offset": lambda s, f: s.__setitem__(64 + 4 * f["nb"], s[64 + 4 * f["nb"]] ^ 1),
 }
