@@ -73,7 +73,16 @@ WORKLOADS = {
     "llama3-8b": ("llama3-8b", None, "Llama-3-8B KV, 8192-token prefill: 32 layers x {K,V} x [8192,8,128] bf16"),
     "qwen3-32b-layer": ("qwen3-32b", 1, "Qwen3-32B KV at 131072 tokens, one layer: {K,V} x [131072,8,128] bf16"),
     "qwen3-30b-a3b-e5m2": ("qwen3-30b-a3b-e5m2", None, "Qwen3-30B-A3B KV, FP8 E5M2: 48 layers x {K,V} x [32768,4,128]"),
+    "stress-uniform-bf16": ("stress-uniform", 1, "escape stress, worst case: one flat bf16 tensor of 2^29 uniformly "
+                                                "random 16-bit patterns (1 GiB)"),
 }
+STRESS_N = 1 << 29        # elements of the stress tensor (1 GiB of bf16)
+STRESS_SAMPLE_N = 1 << 23  # elements of the CPU oracle's sample of it
+
+
+def stress_seed(rank: int = 0) -> int:
+    # the 1 GB uniform-bits case of the escape-stress family (seed 4_000_000 + case); ranks offset
+    return 4_000_000 + kvgen.stress_case(2, len(kvgen.STRESS_RARE_PERCENT) - 1) + 1000 * rank
 
 
 def load_peaks():
@@ -181,6 +190,12 @@ class Workload:
     def __init__(self, name: str, rank: int, world: int, device, layers=None):
         cfg_name, layers_per_step, desc = WORKLOADS[name]
         self.name, self.desc = name, desc
+        if cfg_name == "stress-uniform":
+            self.cfg, self.dtype, self.esize, self.layers = None, 0, 2, [0]
+            self.xs = [kvgen.stress_tensor(STRESS_N, None, stress_seed(rank), device=device)]
+            self.n = [STRESS_N]
+            self.raw_bytes = STRESS_N * 2
+            return
         self.cfg = kvgen.CONFIGS[cfg_name]
         self.dtype = 1 if self.cfg.fp8 else 0
         nl = self.cfg.layers if layers_per_step is None else layers_per_step
@@ -227,6 +242,8 @@ def paged_pools(wl, page_tokens: int, device):
 def run_ours(args, rank, world, device):
     import fp8_kv_cache_exp_b200 as sz
     wl = Workload(args.workload, rank, world, device, args.layers)
+    if wl.cfg is None and (args.mode != "batch" or args.paged or args.transfer or args.layers):
+        raise SystemExit("the stress workload is one flat tensor: batch mode only")
     dt = wl.dtype
     T = len(wl.xs)
     stream = torch.cuda.current_stream()
@@ -252,10 +269,11 @@ def run_ours(args, rank, world, device):
         srcs = [sz.paged(dt, src_pool, tb, page_elems) for tb in src_tabs]
         dsts = [sz.paged(dt, dst_pool, tb, page_elems) for tb in dst_tabs]
         batches = [sz.Batch(dt, None, [outs[i] for i in g], w, p, src_pages=[srcs[i] for i in g],
-                            dst_pages=[dsts[i] for i in g], n=[wl.n[i] for i in g])
+                            dst_pages=[dsts[i] for i in g], n=[wl.n[i] for i in g], raw_blocks=args.raw_blocks)
                    for g, w, p in zip(groups, ws_g, plans_g)]
     else:
-        batches = [sz.Batch(dt, [wl.xs[i] for i in g], [outs[i] for i in g], w, p, decs=[decs[i] for i in g])
+        batches = [sz.Batch(dt, [wl.xs[i] for i in g], [outs[i] for i in g], w, p, decs=[decs[i] for i in g],
+                            raw_blocks=args.raw_blocks)
                    for g, w, p in zip(groups, ws_g, plans_g)]
 
     def plan_all():
@@ -286,12 +304,11 @@ def run_ours(args, rank, world, device):
     for x, d in zip(wl.xs, decs):
         if not torch.equal(x.view(torch.uint8).reshape(-1), d.view(torch.uint8).reshape(-1)):
             raise RuntimeError("round trip mismatch")
-    totals = sz.sz_compressed_sizes(plans)
-    stream_bytes = sum(totals)
-    E_total = 0
-    for i in range(T):
-        h = plans[i].cpu()
-        E_total += int(h[16:24].view(torch.int64).item())
+    # stream lengths and escape-section bytes from the streams' own headers
+    # (with raw blocks the plans hold upper bounds)
+    heads = torch.stack([o[:64] for o in outs]).cpu()
+    stream_bytes = int(heads[:, 40:48].contiguous().view(torch.int64).sum().item())
+    E_total = int(heads[:, 16:24].contiguous().view(torch.int64).sum().item())
 
     if args.reuse:
         def plan_all():  # noqa: F811 -- the timed step reuses the calibration codebooks
@@ -401,6 +418,7 @@ def run_ours(args, rank, world, device):
                    else "own plan per step",
                    "layout": ("paged: %d-token pages, random page order in and out" % args.paged) if args.paged
                    else "contiguous tensors",
+                   "raw_blocks": bool(args.raw_blocks),
                    "raw_bytes_per_rank": wl.raw_bytes, "mode": "one batch" if args.mode == "batch" else "per layer",
                    "l2": "inputs larger than L2 (%.2f GB per step per rank)" % (wl.raw_bytes / 1e9),
                    "parallelism": "replicas" if world == 1 else "dp%d (independent tensors)" % world},
@@ -504,7 +522,7 @@ def run_e2e(args, wl, device):
     outs = [torch.empty(sz.sz_max_compressed_size(dt, n), dtype=torch.uint8, device=device) for n in wl.n]
     stream = torch.cuda.current_stream()
 
-    batch = sz.Batch(dt, dev_in, outs, ws, plans, decs=dev_out)
+    batch = sz.Batch(dt, dev_in, outs, ws, plans, decs=dev_out, raw_blocks=args.raw_blocks)
 
     def step():
         for h, d in zip(host_in, dev_in):
@@ -560,13 +578,20 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def oracle_sample(cfg_name: str, budget_s: float):
-    """Time the CPU oracle (as it stands) on one layer's K and V: plan + encode + decode."""
+def oracle_sample(cfg_name: str, budget_s: float, raw_blocks: bool = False):
+    """Time the CPU oracle (as it stands) on one layer's K and V (the stress
+    workload: a 2^23-element tensor of the same generator): plan + encode + decode."""
     import numpy as np
     import oracle
-    cfg = kvgen.CONFIGS[cfg_name]
-    dt = 1 if cfg.fp8 else 0
-    xs = [kvgen.kv_tensor(cfg, 0, kv) for kv in (0, 1)]
+    if cfg_name == "stress-uniform":
+        dt = 0
+        xs = [kvgen.stress_tensor(STRESS_SAMPLE_N, None, stress_seed())]
+        what = "stress-uniform 2^23 elements"
+    else:
+        cfg = kvgen.CONFIGS[cfg_name]
+        dt = 1 if cfg.fp8 else 0
+        xs = [kvgen.kv_tensor(cfg, 0, kv) for kv in (0, 1)]
+        what = "%s layer 0 K+V" % cfg_name
     raws = [x.contiguous().view(torch.uint8).reshape(-1).numpy() for x in xs]
     nbytes = sum(r.size for r in raws)
     t_enc = t_dec = 0.0
@@ -576,7 +601,7 @@ def oracle_sample(cfg_name: str, budget_s: float):
         for r in raws:
             n = r.size // (2 if dt == 0 else 1)
             t0 = time.perf_counter()
-            s = oracle.encode(dt, r)
+            s = oracle.encode(dt, r, raw_blocks=raw_blocks)
             t1 = time.perf_counter()
             back = oracle.decode(s, n, dt)
             t2 = time.perf_counter()
@@ -591,7 +616,8 @@ def oracle_sample(cfg_name: str, budget_s: float):
     return {
         "value": round(raw_total / (t_enc + t_dec) / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
         "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
-        "sample": "%s layer 0 K+V (%.1f MB raw) x %d rep(s), single-threaded C oracle" % (cfg_name, nbytes / 1e6, reps),
+        "sample": "%s (%.1f MB raw) x %d rep(s), single-threaded C oracle%s" % (
+            what, nbytes / 1e6, reps, ", raw blocks allowed" if raw_blocks else ""),
         "encode_gbs": round(raw_total / t_enc / 1e9, 4), "decode_gbs": round(raw_total / t_dec / 1e9, 4),
         "seconds": round(t_enc + t_dec, 2),
     }
@@ -604,12 +630,13 @@ def run_reference(args, rank, world):
     sample = None
     times = []
     for k in range(args.warmup + args.steps):
-        r = oracle_sample(cfg_name, 0.0)
+        r = oracle_sample(cfg_name, 0.0, args.raw_blocks)
         if k >= args.warmup:
             times.append(r)
         sample = r
     val = statistics.median(t["value"] for t in times)
-    raw = 2 * kvgen.CONFIGS[cfg_name].numel * (1 if kvgen.CONFIGS[cfg_name].fp8 else 2)
+    fp8 = cfg_name != "stress-uniform" and kvgen.CONFIGS[cfg_name].fp8
+    raw = STRESS_SAMPLE_N * 2 if cfg_name == "stress-uniform" else 2 * kvgen.CONFIGS[cfg_name].numel * (1 if fp8 else 2)
     ms = raw / (val * 1e9) * 1e3
     cpu = dict(sample)
     cpu["value"] = val
@@ -617,7 +644,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u8" if kvgen.CONFIGS[cfg_name].fp8 else "u16", "data": "synthetic",
+        "dtype": "u8" if fp8 else "u16", "data": "synthetic",
         "config": {"workload": args.workload, "desc": WORKLOADS[args.workload][2],
                    "sample": cpu["sample"]},
         "cpu_baseline": cpu,
@@ -646,6 +673,8 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the step with direct launches instead of one captured CUDA graph per step "
                          "(per-kernel times always come from direct launches)")
+    ap.add_argument("--raw-blocks", action="store_true",
+                    help="allow raw blocks (header flag): blocks that would expand are stored raw")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -678,7 +707,8 @@ def main():
         if args.transfer:
             res["transfer"] = run_transfer(args, wl, device, res)
         if rank == 0 and world == 1 and args.cpu_baseline_seconds > 0:
-            res["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload][0], args.cpu_baseline_seconds)
+            res["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload][0], args.cpu_baseline_seconds,
+                                                args.raw_blocks)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

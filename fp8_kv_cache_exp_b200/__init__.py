@@ -41,6 +41,7 @@ SZ_HEADER_BYTES = 64
 SZ_BLOCK_ELEMS = 4096
 SZ_MAX_BATCH = 256
 SZ_NOALLOC_MAX_ELEMS = 1 << 27
+SZ_FLAG_RAW_BLOCKS = 1
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitzip.so")
 
@@ -70,6 +71,7 @@ def _load():
         "sz_plan_batched": (i32, [i32, i32, pvp, pu64, vp, sz, vp, vp]),
         "sz_compressed_size": (i32, [vp, pu64, vp]),
         "sz_compressed_sizes": (i32, [i32, vp, pu64, vp]),
+        "sz_plan_set_flags": (i32, [i32, vp, ctypes.c_uint, vp]),
         "sz_encode": (i32, [i32, vp, vp, u64, vp, sz, vp, sz, vp]),
         "sz_encode_batched": (i32, [i32, i32, vp, pvp, pu64, pvp, psz, vp, sz, vp]),
         "sz_encode_reuse": (i32, [i32, vp, vp, u64, vp, sz, vp, vp, sz, vp]),
@@ -213,6 +215,12 @@ def sz_compressed_sizes(plans: torch.Tensor, stream=None):
     return [int(v) for v in out]
 
 
+def sz_plan_set_flags(plans: torch.Tensor, flags: int, stream=None):
+    """Set the header flags (0 or SZ_FLAG_RAW_BLOCKS) of every plan in `plans`."""
+    _check(lib.sz_plan_set_flags(plans.shape[0] if plans.dim() == 2 else 1, _p(plans), int(flags),
+                                 _stream(stream)), "sz_plan_set_flags")
+
+
 def sz_encode(dtype: int, plan: torch.Tensor, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
               stream=None):
     _check(lib.sz_encode(dtype, _p(plan), _p(x), numel_of(x, dtype), _p(out), out.nbytes, _p(ws),
@@ -343,10 +351,13 @@ class Batch:
     """
 
     def __init__(self, dtype: int, xs, outs, ws: torch.Tensor, plans: torch.Tensor, decs=None,
-                 comp_bytes=None, src_pages=None, dst_pages=None, n=None):
+                 comp_bytes=None, src_pages=None, dst_pages=None, n=None, raw_blocks=False):
         """src_pages / dst_pages: paged() descriptors of the inputs / decode outputs
-        (then xs / decs are not read, and n gives the element counts)."""
+        (then xs / decs are not read, and n gives the element counts).
+        raw_blocks: plan() marks the plans so that blocks that would expand are
+        stored raw (SZ_FLAG_RAW_BLOCKS)."""
         outs = list(outs)
+        self._flags = SZ_FLAG_RAW_BLOCKS if raw_blocks else 0
         self._src_pages = None if src_pages is None else _paged_arr(src_pages)
         self._dst_pages = None if dst_pages is None else _paged_arr(dst_pages)
         if src_pages is not None or dst_pages is not None:
@@ -386,9 +397,11 @@ class Batch:
         if self._src_pages is not None:
             _check(lib.sz_plan_paged_batched(self.dtype, self.T, self._src_pages, self._n, self._ws, self._wsb,
                                              self._plans, _stream(stream)), "sz_plan_paged_batched")
-            return
-        _check(lib.sz_plan_batched(self.dtype, self.T, self._in, self._n, self._ws, self._wsb,
-                                   self._plans, _stream(stream)), "sz_plan_batched")
+        else:
+            _check(lib.sz_plan_batched(self.dtype, self.T, self._in, self._n, self._ws, self._wsb,
+                                       self._plans, _stream(stream)), "sz_plan_batched")
+        if self._flags:
+            _check(lib.sz_plan_set_flags(self.T, self._plans, self._flags, _stream(stream)), "sz_plan_set_flags")
 
     def encode(self, stream=None):
         if self._src_pages is not None:

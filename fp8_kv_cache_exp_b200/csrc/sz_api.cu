@@ -130,6 +130,16 @@ sz_status sz_compressed_size(const sz_plan_t *d_plan, uint64_t *h_bytes, cudaStr
     return sz_compressed_sizes(1, d_plan, h_bytes, stream);
 }
 
+sz_status sz_plan_set_flags(int T, sz_plan_t *d_plans, unsigned flags, cudaStream_t stream) {
+    if (T < 1 || T > SZ_MAX_BATCH || !d_plans || !aligned(d_plans, 8)) return SZ_ERR_INVALID_ARG;
+    if (flags & ~unsigned(SZ_FLAG_RAW_BLOCKS)) return SZ_ERR_INVALID_ARG;
+    // byte 39 of each of the T consecutive 64-byte plans: one strided memset
+    if (cudaMemset2DAsync(reinterpret_cast<uint8_t *>(d_plans) + 39, sizeof(sz_plan_t), int(flags), 1, size_t(T),
+                          stream) != cudaSuccess)
+        return SZ_ERR_CUDA;
+    return SZ_OK;
+}
+
 namespace {
 
 // Ordinary encode (plans are the tensors' own) or codebook reuse (plans give

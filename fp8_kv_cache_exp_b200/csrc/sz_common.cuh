@@ -24,6 +24,7 @@ constexpr uint32_t kBlockLog2 = 12;
 constexpr uint32_t kBlock = 1u << kBlockLog2;  // elements per escape-offset block (= one tile)
 constexpr uint32_t kCodes = 15;                // codes 0..14 name codebook entries
 constexpr uint32_t kEscape = 15;               // code 15 marks an escaped exponent
+constexpr uint32_t kFlagRawBlocks = 1;         // header byte 39, bit 0: raw blocks allowed
 constexpr int kTileThreads = 256;              // threads per encode/decode tile CTA
 constexpr int kSmallBatch = 8;                 // parameter blocks sized for <= 8 tensors ...
 constexpr int kLargeBatch = SZ_MAX_BATCH;      // ... or for up to SZ_MAX_BATCH tensors
@@ -74,6 +75,16 @@ template <> struct Dt<SZ_FP8_E5M2> {
     static constexpr int kBins = 32;       // 5-bit exponent
     static constexpr int kElemBytes = 1;
 };
+
+// Escape-section bytes of a raw block of m elements: the exponent bits above
+// the low four, which its code nibbles hold (four per BF16 element, one per
+// E5M2 element).  With raw blocks allowed, a block whose escapes would fill at
+// least this many bytes is stored raw, and a coded block has fewer escapes, so
+// its offsets-table count tells which it is.
+template <int DT>
+__host__ __device__ constexpr uint32_t raw_block_bytes(uint32_t m) {
+    return DT == SZ_BF16 ? (m + 1) / 2 : (m + 7) / 8;
+}
 
 // Section offsets of a stream with n elements and E escapes.
 struct Layout {
@@ -430,7 +441,7 @@ __device__ __forceinline__ uint32_t pick4(uint32_t w0, uint32_t w1, uint32_t w2,
 struct Header {
     uint32_t magic, vtag;  // vtag = version | dtype << 16 | block_log2 << 24
     uint64_t n, E, total;
-    uint32_t cbw[4];       // cb[0..14] in bytes 0..14, byte 15 zero
+    uint32_t cbw[4];       // cb[0..14] in bytes 0..14, byte 15 the flags
 };
 
 __device__ inline Header load_header(const uint8_t *h) {

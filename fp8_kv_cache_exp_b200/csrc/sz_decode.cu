@@ -81,6 +81,7 @@ struct DFrag {
 struct WarpStream {
     int t;                        // tensor, -1 if none yet
     bool ok;                      // header passed every check
+    bool raw_ok;                  // the stream may hold raw blocks (header flag)
     uint32_t nb;                  // 4096-element blocks
     uint64_t n, E;
     uint64_t code, pa, pb, esc;   // section offsets in the stream
@@ -165,7 +166,7 @@ __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, in
     const uint64_t total = uint64_t(w[10]) | (uint64_t(w[11]) << 32);
     const uint32_t cbw[4] = {w[6], w[7], w[8], w[9]};
     bool ok = w[0] == kMagic && (w[1] & 0xFF00FFFFu) == (header_vtag(DT) & 0xFF00FFFFu) &&
-              ((w[1] >> 16) & 0xFFu) == uint32_t(DT) && hn == n && E <= n && (w[9] >> 24) == 0 &&
+              ((w[1] >> 16) & 0xFFu) == uint32_t(DT) && hn == n && E <= n && ((w[9] >> 24) & ~kFlagRawBlocks) == 0 &&
               total == stream_layout(DT, n, E).total && total <= p.comp_bytes[t];
     // codebook: 15 distinct values inside the exponent range
     bool cb_ok = true;
@@ -191,6 +192,7 @@ __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, in
     const Layout L = stream_layout(DT, n, ok ? E : 0);
     ws.t = t;
     ws.ok = ok;
+    ws.raw_ok = ((w[9] >> 24) & kFlagRawBlocks) != 0;
     ws.nb = uint32_t(L.nb);
     ws.n = n;
     ws.E = E;
@@ -199,9 +201,10 @@ __device__ __forceinline__ void warp_open_stream(const DecodeParams<MAXB> &p, in
     ws.pb = L.plane[1];
     ws.esc = L.esc;
     // E5M2 exponents are below 32, so every byte of the x4 table stays below
-    // 128: a selector nibble with its top bit set reads as zero (see prmt)
+    // 128: a selector nibble with its top bit set reads as zero (see prmt).
+    // Byte 15 (code 15) is 0: the flags byte is masked off.
 #pragma unroll
-    for (int i = 0; i < 4; ++i) ws.xt[i] = ok ? (cbw[i] << 2) : 0u;
+    for (int i = 0; i < 4; ++i) ws.xt[i] = ok ? ((i == 3 ? (cbw[i] & 0x00FFFFFFu) : cbw[i]) << 2) : 0u;
 }
 
 // Section offsets of a tensor's stream; they depend on n only.
@@ -377,6 +380,67 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
     }
 }
 
+// Decode one step of a raw block: the code nibbles are the low four exponent
+// bits; hs points at this lane's share of the block's high bits in the escape
+// section (BF16: a high nibble per element, E5M2: bit 4 per element).  Only
+// `valid` elements exist (LE for a full step).  Rare by construction: plain
+// per-element code.
+template <int DT, bool PARTIAL, bool CHECKED>
+__device__ __forceinline__ void raw_step_body(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid,
+                                              bool store) {
+    constexpr int LE = DGeo<DT>::LE;
+    const int hbytes = (DT == SZ_BF16) ? (valid + 1) / 2 : (valid + 7) / 8;
+    uint32_t hi = 0;
+    for (int b = 0; b < hbytes; ++b) hi |= uint32_t(hs[b]) << (8 * b);
+    uint32_t o[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < LE; ++j) {
+        const uint32_t lo = (((j < 8) ? f.c0 : f.c1) >> (4 * (j & 7))) & 0xFu;
+        if constexpr (DT == SZ_BF16) {
+            const uint32_t e = lo | (((hi >> (4 * j)) & 0xFu) << 4);
+            const uint32_t sm = (((j < 4) ? f.a : f.b) >> (8 * (j & 3))) & 0xFFu;
+            const uint32_t v = ((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu);
+            o[j >> 1] |= v << (16 * (j & 1));
+        } else {
+            const uint32_t e = lo | (((hi >> j) & 1u) << 4);
+            const uint32_t sg = (f.a >> j) & 1u, mt = (f.b >> (2 * j)) & 3u;
+            o[j >> 2] |= ((sg << 7) | (e << 2) | mt) << (8 * (j & 3));
+        }
+    }
+    if (CHECKED && !store) {
+        // an output page outside the pool: nothing is written
+    } else if (!PARTIAL) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else if constexpr (DT == SZ_BF16) {
+        for (int j = 0; j < valid; ++j) reinterpret_cast<uint16_t *>(dst)[j] = uint16_t(o[j >> 1] >> (16 * (j & 1)));
+    } else {
+        for (int j = 0; j < valid; ++j) dst[j] = uint8_t(o[j >> 2] >> (8 * (j & 3)));
+    }
+}
+
+template <int DT, bool PARTIAL, bool CHECKED>
+__device__ __noinline__ void raw_step_outlined(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid,
+                                               bool store) {
+    raw_step_body<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
+}
+
+// The raw step is a call in the BF16 kernels and inline in the E5M2 ones: each
+// leaves the coded path faster that way (measured).
+template <int DT, bool PARTIAL, bool CHECKED = false>
+__device__ __forceinline__ void decode_step_raw(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid,
+                                                bool store = true) {
+    if constexpr (DT == SZ_BF16) raw_step_outlined<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
+    else raw_step_body<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
+}
+
+// This lane's high bits of step `it` of a raw block within the block's escape
+// section esc_g.
+template <int DT>
+__device__ __forceinline__ const uint8_t *raw_high(const uint8_t *esc_g, int it) {
+    const uint32_t local = uint32_t(it) * 32 * DGeo<DT>::LE + (threadIdx.x & 31) * DGeo<DT>::LE;
+    return esc_g + ((DT == SZ_BF16) ? local / 2 : local / 8);
+}
+
 // Offsets-table entries of a block and their checks.
 struct BlockEsc {
     uint32_t lo, hi;
@@ -547,6 +611,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
             constexpr int EB = Dt<DT>::kElemBytes;
             uint8_t *out = p.out[t] + (uint64_t(blk) * kBlock + uint64_t(lane) * G::LE) * EB;
             const bool full = (uint64_t(blk) + 1) * kBlock <= ws.n;
+            // a raw block: its count is exactly raw_block_bytes (a coded block has fewer escapes)
+            const bool raw = ok && ws.raw_ok &&
+                             cnt == raw_block_bytes<DT>(full ? kBlock : uint32_t(ws.n - uint64_t(blk) * kBlock));
             // paged output: lane q < G::kUnits looks up where unit q of the block goes
             uint64_t qoff = 0;
             if constexpr (PAGED) {
@@ -577,12 +644,24 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                             const bool store = off != kBadOffset;
                             uint8_t *out_q = p.out[t] + off + uint64_t(lane) * G::LE * EB;
                             if (!store && lane == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
+                            if (raw) {
+                                for (int it = 0; it < G::QIT; ++it)
+                                    decode_step_raw<DT, false, true>(read_stage<DT, G>(st_addr, it),
+                                                                     raw_high<DT>(esc_g, q * G::QIT + it),
+                                                                     out_q + it * 512, G::LE, store);
+                            } else {
 #pragma unroll
-                            for (int it = 0; it < G::QIT; ++it) {
-                                const DFrag f = read_stage<DT, G>(st_addr, it);
-                                decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE, running,
-                                                             esc_reg, esc_g, cnt, bad, store);
+                                for (int it = 0; it < G::QIT; ++it) {
+                                    const DFrag f = read_stage<DT, G>(st_addr, it);
+                                    decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE,
+                                                                 running, esc_reg, esc_g, cnt, bad, store);
+                                }
                             }
+                        } else if (raw) {
+                            for (int it = 0; it < G::QIT; ++it)
+                                decode_step_raw<DT, false>(read_stage<DT, G>(st_addr, it),
+                                                           raw_high<DT>(esc_g, q * G::QIT + it),
+                                                           out + (q * G::QIT + it) * 512, G::LE);
                         } else {
 #pragma unroll
                             for (int it = 0; it < G::QIT; ++it) {
@@ -606,8 +685,13 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                                     dst = p.out[t] + off;
                                     if (!store) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
                                 }
-                                decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg, esc_g,
-                                                            cnt, bad, store);
+                                if (raw)
+                                    decode_step_raw<DT, true, true>(f, raw_high<DT>(esc_g, it), dst, valid, store);
+                                else
+                                    decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg,
+                                                                esc_g, cnt, bad, store);
+                            } else if (raw) {
+                                decode_step_raw<DT, true>(f, raw_high<DT>(esc_g, it), out + it * 512, valid);
                             } else {
                                 decode_step<DT, true>(f, tab_addr, ws.xt, out + it * 512, valid, running, esc_reg,
                                                       esc_g, cnt, bad);
@@ -617,6 +701,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                 }
                 __syncwarp();  // the stage just read may be refilled from here on
             }
+            if (raw) running = cnt;  // a raw block's high bits fill its count exactly
             if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
             if (lane == 0) {
                 const uint32_t g = p.block_begin[t] + blk;

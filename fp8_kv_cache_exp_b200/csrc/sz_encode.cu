@@ -147,12 +147,15 @@ __device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t 
     return true;
 }
 
-// The plan's codebook: 15 distinct values inside the exponent range and a zero
-// pad byte (one lane per entry; warp-wide).
+// Header flags (byte 39).
+__device__ __forceinline__ uint32_t header_flags(const Header &H) { return H.cbw[3] >> 24; }
+
+// The plan's codebook: 15 distinct values inside the exponent range, and
+// flags no other than kFlagRawBlocks (one lane per entry; warp-wide).
 template <int DT>
 __device__ __forceinline__ bool codebook_ok(const Header &H) {
     const int lane = threadIdx.x & 31;
-    bool ok = (H.cbw[3] >> 24) == 0;
+    bool ok = (header_flags(H) & ~kFlagRawBlocks) == 0;
     if (lane < int(kCodes)) {
         const uint32_t v = cb_byte(H.cbw, lane);
         ok = ok && v < uint32_t(Dt<DT>::kBins);
@@ -467,6 +470,51 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     return running;
 }
 
+// One warp stores block blk raw (raw blocks allowed and its escapes would
+// fill at least raw_block_bytes): the low four bits of each exponent
+// overwrite the block's code nibbles, the remaining bits go to the escape
+// section at byte d (BF16: high nibbles, element j of the block in nibble j%2
+// of byte j/2; E5M2: bit 4 at bit j%8 of byte j/8), bytes at or past bound
+// not written.  Planes are as coded.  Rare by construction (data that the
+// codebook misses), so this reads its input again from global memory.
+template <int DT, bool PAGED>
+__device__ void raw_block(const uint8_t *in, const PageRef &pr, uint64_t n, uint64_t blk, const Layout &L,
+                          uint8_t *out, uint64_t d, uint64_t bound) {
+    using G = Geo<DT>;
+    const int lane = threadIdx.x & 31;
+    const uint64_t e_lane = blk * kBlock + uint64_t(lane) * G::LE;
+    const bool paged = PAGED && pr.pages != nullptr;
+    uint8_t *code = out + L.code + e_lane / 2;
+#pragma unroll 1
+    for (int it = 0; it < G::IT; ++it) {
+        const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
+        const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+        if (valid <= 0) continue;
+        const uint64_t e = e_lane + uint64_t(it) * 32 * G::LE;
+        const uint64_t off = paged ? elem_offset<Dt<DT>::kElemBytes>(pr, e) : e * Dt<DT>::kElemBytes;
+        const uint4 v = off != kBadOffset ? load_step<DT>(in + off, valid) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t lo[2] = {0, 0}, hi = 0;
+#pragma unroll
+        for (int j = 0; j < G::LE; ++j) {
+            uint32_t x;
+            if constexpr (DT == SZ_BF16) x = (w[j >> 1] >> (16 * (j & 1) + 7)) & 0xFFu;
+            else x = (w[j >> 2] >> (8 * (j & 3) + 2)) & 0x1Fu;
+            lo[j >> 3] |= (x & 0xFu) << (4 * (j & 7));
+            if constexpr (DT == SZ_BF16) hi |= (x >> 4) << (4 * j);
+            else hi |= (x >> 4) << j;
+        }
+        // code nibbles: the same bytes code_step wrote for this lane
+        store_bytes(code + it * EStride<DT>::code, lo[0], lo[1], (valid + 1) / 2);
+        // high bits: this lane's share of the block's raw_block_bytes
+        const uint32_t local = uint32_t(it) * 32 * G::LE + uint32_t(lane) * G::LE;  // within the block
+        const uint64_t h0 = d + ((DT == SZ_BF16) ? local / 2 : local / 8);
+        const int hbytes = (DT == SZ_BF16) ? (valid + 1) / 2 : (valid + 7) / 8;
+        for (int b = 0; b < hbytes; ++b)
+            if (h0 + b < bound) out[h0 + b] = uint8_t(hi >> (8 * b));
+    }
+}
+
 // The warp's input ring: units (Units below) of the chunk being coded,
 // stage = unit % kRing; units of a partial (last) block are not copied and
 // are read from global memory instead.
@@ -570,11 +618,14 @@ __device__ __forceinline__ ChunkGeo chunk_geo(const EncodeParams<MAXB> &p, uint3
 
 // One warp codes a chunk: planes and codes go out, escapes are staged in
 // esc[slot] (element order) with per-block offsets in blk_off[slot].  Between
-// blocks it calls between().  Returns the chunk's escape count, or
+// blocks it calls between().  Returns the chunk's escape-section bytes, or
 // 0xFFFFFFFF if the plan does not fit the data (reported; nothing to finish).
+// With raw blocks allowed, bit k of *raw is set for each block k of the chunk
+// that is to be stored raw; it counts raw_block_bytes.
 template <int DT, int MAXB, bool PAGED, typename Between>
 __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
-                               WarpShared &W, RingState &R, int &plan_tensor, bool *lost, Between between) {
+                               WarpShared &W, RingState &R, int &plan_tensor, bool *lost, uint32_t *raw,
+                               Between between) {
     const int lane = threadIdx.x & 31;
     const uint8_t *in = p.in[g.t];
     uint8_t *out = p.out[g.t];
@@ -591,6 +642,8 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
         return 0xFFFFFFFFu;  // every chunk of this tensor takes this branch: no look-back waits on it
     }
     const Layout L = stream_layout(DT, n, p.reuse ? 0 : H.E);  // section starts do not depend on E
+    const bool raw_ok = (header_flags(H) & kFlagRawBlocks) != 0;
+    *raw = 0;
 
     using G = Geo<DT>;
     using UN = Units<DT, PAGED>;
@@ -651,6 +704,13 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
             }
             __syncwarp();  // the stage just read may be refilled from here on
         }
+        if (raw_ok) {
+            const uint32_t m = full ? kBlock : uint32_t(n - blk * kBlock);
+            if (blk_run >= raw_block_bytes<DT>(m)) {
+                blk_run = raw_block_bytes<DT>(m);
+                *raw |= 1u << k;
+            }
+        }
         running += blk_run;
         between();
     }
@@ -660,14 +720,17 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
 
 // Once the chunk's offset excl is known: its offsets-table entries, its
 // escapes (from the stage, or re-coded from the input when they overflowed
-// it -- the warp's code table is then still the chunk's), and the stream
-// frame if it is the tensor's last chunk.
+// it or the chunk has raw blocks -- the warp's code table is then still the
+// chunk's), and the stream frame if it is the tensor's last chunk.
 template <int DT, int MAXB, bool PAGED>
 __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
-                             uint32_t total, const Lookback &lb, WarpShared &W) {
+                             uint32_t total, uint32_t raw, const Lookback &lb, WarpShared &W) {
     const int lane = threadIdx.x & 31;
     const Header H = load_header(p.plans + 64 * size_t(g.t));
     const bool reuse = p.reuse != 0;
+    // the plan's E counts every escape; raw blocks store fewer bytes, so with
+    // raw blocks allowed E is known only at the end, as with a reused codebook
+    const bool raw_ok = (header_flags(H) & kFlagRawBlocks) != 0;
     const Layout L = stream_layout(DT, g.n, reuse ? 0 : H.E);
     uint8_t *out = p.out[g.t];
     const uint32_t excl = lb.excl;
@@ -676,14 +739,14 @@ __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const Ch
         if (lb.flags & kLbTimedOut) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
         if (!reuse) {
             if (uint64_t(excl) + total > H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
-            if (last && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
+            if (!raw_ok && last && uint64_t(excl) + total != H.E) set_error(p.ctl, SZ_ERR_PLAN_MISMATCH, job);
         }
     }
     if (lane < g.nbk) *reinterpret_cast<uint32_t *>(out + 64 + 4 * (g.b0 + lane)) = excl + W.blk_off[slot][lane];
     // escapes past the stream's end (ordinary encode) or the buffer's (reuse) are not written
     const uint64_t bound = reuse ? p.cap[g.t] : L.total;
     const uint64_t dst = L.esc + excl;
-    if (total <= kWarpStage) {
+    if (total <= kWarpStage && raw == 0) {
         for (uint32_t x = lane; x < total; x += 32)
             if (dst + x < bound) out[dst + x] = W.esc[slot][x];
     } else {
@@ -691,14 +754,19 @@ __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const Ch
 #pragma unroll 1
         for (int k = 0; k < g.nbk; ++k) {
             const uint64_t d = dst + W.blk_off[slot][k];
-            code_block<DT, false, PAGED>(lut, p.in[g.t], p.pg[g.t], g.n, g.b0 + k, L, out, [&](uint32_t r, uint32_t e) {
-                if (d + r < bound) out[d + r] = uint8_t(e);
-            });
+            if ((raw >> k) & 1u) {
+                raw_block<DT, PAGED>(p.in[g.t], p.pg[g.t], g.n, g.b0 + k, L, out, d, bound);
+            } else {
+                code_block<DT, false, PAGED>(lut, p.in[g.t], p.pg[g.t], g.n, g.b0 + k, L, out,
+                                             [&](uint32_t r, uint32_t e) {
+                                                 if (d + r < bound) out[d + r] = uint8_t(e);
+                                             });
+            }
         }
     }
     if (last) {
-        // the tensor's escape count is now known: excl + total
-        const uint64_t E = reuse ? uint64_t(excl) + total : H.E;
+        // the tensor's escape-section length is now known: excl + total
+        const uint64_t E = (reuse || raw_ok) ? uint64_t(excl) + total : H.E;
         const uint64_t stream_total = stream_layout(DT, g.n, E).total;
         if (reuse && stream_total > p.cap[g.t] && lane == 0) set_error(p.ctl, SZ_ERR_BUFFER_TOO_SMALL, job);
         write_stream_frame(out, L, header_word<DT>(lane, g.n, E, stream_total, H.cbw), E);
@@ -764,7 +832,7 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
         if (!pend.valid) return;
         const ChunkGeo pg = chunk_geo<MAXB, LG>(p, pend.job);
         if (lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, block)) {
-            finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, pend.lb, W);
+            finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W);
             pend.valid = false;
         }
     };
@@ -781,7 +849,8 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
         const ChunkGeo g = chunk_geo<MAXB, LG>(p, job);
         const int slot = pend.valid ? (pend.slot ^ 1) : 0;
         bool lost = false;
-        const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost,
+        uint32_t raw = 0;
+        const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost, &raw,
                                                     [&]() { settle(false); });
         if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
         if (total == 0xFFFFFFFFu) continue;  // plan rejected for this tensor
@@ -789,9 +858,10 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
         Lookback lb;
         lookback_start(lb, st, g.chunk, total, tag);
         settle(true);  // at most one chunk waits for its offset
-        if (total > kWarpStage || lookback_advance(lb, st, g.chunk, total, tag, false)) {
+        // chunks that re-read their input (escape overflow, raw blocks) finish at once
+        if (total > kWarpStage || raw != 0 || lookback_advance(lb, st, g.chunk, total, tag, false)) {
             lookback_advance(lb, st, g.chunk, total, tag, true);
-            finish_chunk<DT, MAXB, PAGED>(p, job, g, slot, total, lb, W);
+            finish_chunk<DT, MAXB, PAGED>(p, job, g, slot, total, raw, lb, W);
         } else {
             pend.valid = true;
             pend.job = job;

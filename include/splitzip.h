@@ -16,7 +16,7 @@
  *
  *   [0,64)  header: u32 magic 0x564B5A53 ("SZKV"), u16 version 1, u8 dtype,
  *           u8 block_log2 = 12, u64 n, u64 E (escapes), u8 cb[15] (codebook:
- *           exponent of code c), u8 0, u64 total_bytes, 16 zero bytes
+ *           exponent of code c), u8 flags, u64 total_bytes, 16 zero bytes
  *   [64, 64+4(nb+1))  u32 offsets[nb+1], nb = ceil(n/4096): escapes before
  *           each 4096-element block (exclusive prefix), offsets[nb] = E
  *   then, each section starting at the next multiple of 256 bytes:
@@ -29,7 +29,22 @@
  *   Codebook: the 15 exponent values ranked first by (count descending,
  *   value ascending); code c names cb[c]; code 15 = escape, whose exponent
  *   (zero-extended to a byte for E5M2) is the next byte of the escape stream,
- *   in element order.  The stream is a pure function of the input.
+ *   in element order.  The stream is a pure function of the input and the
+ *   flags.
+ *
+ *   Header byte 39 holds the flags, 0 unless raw blocks are allowed.  With
+ *   SZ_FLAG_RAW_BLOCKS, a block of m elements whose escapes would fill at
+ *   least K = ceil(m/2) bytes (BF16) or ceil(m/8) bytes (E5M2) is stored raw
+ *   instead: its code nibbles hold the low four bits of each exponent, and K
+ *   escape-section bytes hold the rest (BF16: the high nibble of block
+ *   element j's exponent in nibble j%2 of byte j/2; E5M2: bit 4 at bit j%8 of
+ *   byte j/8).  The offsets table counts K for it; a coded block always has
+ *   fewer escapes than K, so the count tells the two apart.  E is then the
+ *   escape section's length.  A raw block costs exactly its raw bytes, so no
+ *   block expands: a stream is at most the raw tensor plus header, table
+ *   and section padding (uniform random bits would otherwise take some 19.5
+ *   bits per BF16 element).  The project page describes no such fallback;
+ *   it is this format's own extension for data the codebook does not fit.
  *
  * Conventions for every call:
  *   - Pointers named d_* are device pointers on the current device; the
@@ -91,6 +106,7 @@ typedef enum { SZ_BF16 = 0, SZ_FP8_E5M2 = 1 } sz_dtype;
 #define SZ_BLOCK_ELEMS 4096
 #define SZ_MAX_BATCH 256
 #define SZ_FORMAT_VERSION 1
+#define SZ_FLAG_RAW_BLOCKS 1u /* header byte 39, bit 0: blocks that would expand are stored raw */
 
 /* A plan is the 64-byte stream header of the tensor it was made for:
  * codebook, n, E and total_bytes.  It lives in device memory. */
@@ -182,6 +198,17 @@ sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
                             const size_t *out_cap, void *d_ws, size_t ws_bytes,
                             cudaStream_t stream);
 
+/* Set the header flags of T consecutive plans (byte 39; 0 or
+ * SZ_FLAG_RAW_BLOCKS), stream-ordered after the sz_plan* call that wrote
+ * them (a plan call writes flags 0).  Encoding with a plan, or with it as a
+ * reused codebook, then allows raw blocks; the stream records the flag and
+ * sz_decode reads it.  With raw blocks the plan's E and total_bytes are upper
+ * bounds (a raw block stores fewer bytes than its escapes would): out_cap
+ * checks use them, and the stream's own header (bytes 16..23 and 40..47) holds
+ * the exact E and length.  SZ_ERR_INVALID_ARG for other flags, T out of
+ * range or a null/misaligned pointer. */
+sz_status sz_plan_set_flags(int T, sz_plan_t *d_plans, unsigned flags, cudaStream_t stream);
+
 /* Codebook reuse: encode with the codebook of a plan made earlier -- for
  * another layer, or for the same tensor at an earlier step -- without a new
  * histogram pass.  Any codebook keeps the stream lossless: every exponent
@@ -190,9 +217,9 @@ sz_status sz_encode_batched(sz_dtype dtype, int T, const sz_plan_t *d_plans,
  * stream that sz_decode reads; its header records the given codebook and the
  * escape count E that codebook leaves for this data.
  *
- * Only the codebook bytes (plan bytes 24..39, 15 distinct values of the
- * dtype's exponent range, byte 39 zero) are read from d_codebook; its n, E
- * and total are ignored.  An invalid codebook is reported as
+ * Only the codebook bytes (plan bytes 24..38, 15 distinct values of the
+ * dtype's exponent range) and the flags (byte 39, see sz_plan_set_flags) are
+ * read from d_codebook; its n, E and total are ignored.  An invalid codebook is reported as
  * SZ_ERR_PLAN_MISMATCH on the device error word and nothing is written.
  *
  * out_cap must hold at least sz_stream_bytes(dtype, n, 0) (checked here).

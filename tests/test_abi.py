@@ -73,3 +73,17 @@ def test_status_strings():
     assert sz.sz_status_string(0) == "ok"
     assert "corrupt" in sz.sz_status_string(4)
     assert sz.sz_status_string(99) == "unknown status"
+
+
+def test_plan_set_flags_host_checks(lib):
+    """Rejected on the host, before any CUDA call: no plans, too many, a null or
+    misaligned pointer, unknown flag bits."""
+    f = lib.sz_plan_set_flags
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    assert f(0, fake, 1, None) == 1
+    assert f(257, fake, 1, None) == 1
+    assert f(1, None, 1, None) == 1
+    assert f(1, fake + 4, 1, None) == 1
+    assert f(1, fake, 2, None) == 1

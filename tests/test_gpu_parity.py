@@ -70,14 +70,17 @@ def test_golden_streams_on_gpu():
     for path in oracle_pins.golden_files():
         dtype, raw, expect = oracle_pins.load_golden(path)
         cb = oracle_pins.golden_codebook(path)
+        flags = oracle_pins.golden_flags(path)
         if cb is None:
+            assert flags == 0
             plan, stream = gpu_encode(dtype, from_raw(raw, dtype))
-        else:  # a codebook-reuse fixture: encode with the given codebook
+        else:  # a codebook-reuse fixture: encode with the given codebook (and flags)
             x = from_raw(raw, dtype)
             n = m.numel_of(x, dtype)
             ws = m.new_workspace(dtype, [n])
             h = np.zeros((1, 64), dtype=np.uint8)
             h[0, 24:39] = cb
+            h[0, 39] = flags
             out = torch.full((m.sz_max_compressed_size(dtype, n),), 0xA5, dtype=torch.uint8, device="cuda")
             m.sz_encode_reuse(dtype, torch.from_numpy(h).cuda(), x, out, ws)
             assert m.sz_last_device_status(ws) == 0
