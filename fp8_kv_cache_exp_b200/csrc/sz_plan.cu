@@ -38,22 +38,27 @@ struct PlanCfg {
     static constexpr uint32_t kItemElems = kItemBytes / kElemBytes;
 };
 
-// Count the elements of one 16-byte vector.  col = this thread's column
-// (s_cols + tid % (NT/2)); inc = its half (1 or 1 << 16).
+// Add inc to the shared-memory word at addr (no return value needed).
+__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t inc) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(inc) : "memory");
+}
+
+// Count the elements of one 16-byte vector.  col = shared address of this
+// thread's column (s_cols + tid % (NT/2)); inc = its half (1 or 1 << 16).
 template <int DT, int NT>
-__device__ __forceinline__ void count_vec(uint32_t *col, uint32_t inc, uint4 v) {
-    constexpr int kRow = NT / 2;  // words per exponent value
+__device__ __forceinline__ void count_vec(uint32_t col, uint32_t inc, uint4 v) {
+    constexpr uint32_t kRowBytes = NT / 2 * 4;  // bytes per exponent value
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         if constexpr (DT == SZ_BF16) {
             // two elements per word: exponent bits 7..14 and 23..30
-            atomicAdd(col + ((w[k] >> 7) & 0xFFu) * kRow, inc);
-            atomicAdd(col + ((w[k] >> 23) & 0xFFu) * kRow, inc);
+            red_shared_add(col + ((w[k] >> 7) & 0xFFu) * kRowBytes, inc);
+            red_shared_add(col + ((w[k] >> 23) & 0xFFu) * kRowBytes, inc);
         } else {
             // four elements per word: exponent bits 2..6 of each byte
 #pragma unroll
-            for (int b = 0; b < 4; ++b) atomicAdd(col + ((w[k] >> (8 * b + 2)) & 0x1Fu) * kRow, inc);
+            for (int b = 0; b < 4; ++b) red_shared_add(col + ((w[k] >> (8 * b + 2)) & 0x1Fu) * kRowBytes, inc);
         }
     }
 }
@@ -69,39 +74,55 @@ __device__ __forceinline__ uint32_t exponent_scalar(const uint8_t *in, uint64_t 
 }
 
 // Count elements [a, b) of one tensor (a is a multiple of the vector size).
+// Batches of U vectors per thread are software-pipelined: the next batch is
+// loaded while the current one is counted.  Only the last, partial batch needs
+// bounds checks.
 template <int DT, int NT>
-__device__ void count_range(uint32_t *col, uint32_t inc, const uint8_t *in, uint64_t a, uint64_t b) {
+__device__ void count_range(uint32_t col, uint32_t inc, const uint8_t *in, uint64_t a, uint64_t b) {
     using C = PlanCfg<DT>;
     constexpr int U = kPlanUnroll;
-    const uint4 *src = reinterpret_cast<const uint4 *>(in) + a / C::kVecElems;
-    const uint64_t nvec = (b - a) / C::kVecElems;
+    constexpr uint32_t kBatch = uint32_t(U) * NT;
     const int tid = threadIdx.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(in) + a / C::kVecElems + tid;
+    const uint32_t nvec = uint32_t((b - a) / C::kVecElems);  // < 2^29: sub-ranges are short
+    const uint32_t full = nvec / kBatch;                       // batches with every vector in range
+    auto load_checked = [&](uint4 (&dst)[U], uint32_t base) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t k = base + uint32_t(tid) + uint32_t(u) * NT;
+            dst[u] = k < nvec ? __ldg(src + (base + uint32_t(u) * NT)) : make_uint4(0, 0, 0, 0);
+        }
+    };
     uint4 cur[U];
+    if (full > 0) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint64_t k = uint64_t(tid) + uint64_t(u) * NT;
-        cur[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < U; ++u) cur[u] = __ldg(src + uint32_t(u) * NT);
+    } else {
+        load_checked(cur, 0);
     }
-    for (uint64_t base = 0; base < nvec; base += uint64_t(U) * NT) {
+    for (uint32_t bi = 0; bi < full; ++bi) {
         uint4 nxt[U];
-        const uint64_t nbase = base + uint64_t(U) * NT;
+        const uint32_t nbase = (bi + 1) * kBatch;
+        if (bi + 1 < full) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint64_t k = nbase + tid + uint64_t(u) * NT;
-            nxt[u] = k < nvec ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < U; ++u) nxt[u] = __ldg(src + (nbase + uint32_t(u) * NT));
+        } else {
+            load_checked(nxt, nbase);
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint64_t k = base + tid + uint64_t(u) * NT;
-            if (k < nvec) count_vec<DT, NT>(col, inc, cur[u]);
-        }
+        for (int u = 0; u < U; ++u) count_vec<DT, NT>(col, inc, cur[u]);
 #pragma unroll
         for (int u = 0; u < U; ++u) cur[u] = nxt[u];
     }
+    // the partial batch (already loaded, zero past the end)
+    const uint32_t tail = full * kBatch;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+        if (tail + uint32_t(tid) + uint32_t(u) * NT < nvec) count_vec<DT, NT>(col, inc, cur[u]);
     // ragged end (< one vector): thread 0 counts it element by element
     if (tid == 0) {
-        for (uint64_t i = a + nvec * C::kVecElems; i < b; ++i)
-            atomicAdd(col + exponent_scalar<DT>(in, i) * (NT / 2), inc);
+        for (uint64_t i = a + uint64_t(nvec) * C::kVecElems; i < b; ++i)
+            red_shared_add(col + exponent_scalar<DT>(in, i) * (NT / 2 * 4), inc);
     }
 }
 
@@ -115,7 +136,7 @@ constexpr uint32_t kPageCache = 4096;
 // once wherever they lie in the pool.  A page id outside the pool sets *bad and
 // that page is not counted.
 template <int DT, int NT>
-__device__ void count_range_paged(uint32_t *col, uint32_t inc, const uint8_t *pool, const PageRef &pr,
+__device__ void count_range_paged(uint32_t col, uint32_t inc, const uint8_t *pool, const PageRef &pr,
                                   uint64_t a, uint64_t b, int32_t *s_ids, bool *bad) {
     using C = PlanCfg<DT>;
     constexpr int U = kPlanUnroll;
@@ -173,7 +194,7 @@ __device__ void count_range_paged(uint32_t *col, uint32_t inc, const uint8_t *po
                 *bad = true;
                 continue;
             }
-            atomicAdd(col + exponent_scalar<DT>(pool + off, 0) * (NT / 2), inc);
+            red_shared_add(col + exponent_scalar<DT>(pool + off, 0) * (NT / 2 * 4), inc);
         }
     }
 }
@@ -270,7 +291,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
     __shared__ uint32_t s_words[16];
     __shared__ uint32_t s_last;
     const int tid = threadIdx.x;
-    uint32_t *col = s_cols + (tid % (NT / 2));
+    const uint32_t col = smem_u32(s_cols + (tid % (NT / 2)));
     const uint32_t inc = 1u << (16 * (tid / (NT / 2)));
 
     // Plans of empty tensors: codebook of the 15 smallest values, E = 0.
