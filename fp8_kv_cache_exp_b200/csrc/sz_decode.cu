@@ -418,19 +418,18 @@ __device__ __forceinline__ void raw_step_body(const DFrag &f, const uint8_t *hs,
     }
 }
 
-template <int DT, bool PARTIAL, bool CHECKED>
-__device__ __noinline__ void raw_step_outlined(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid,
-                                               bool store) {
-    raw_step_body<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
+template <int DT, bool PARTIAL>
+__device__ __noinline__ void raw_step_outlined(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid) {
+    raw_step_body<DT, PARTIAL, false>(f, hs, dst, valid, true);
 }
 
-// The raw step is a call in the BF16 kernels and inline in the E5M2 ones: each
-// leaves the coded path faster that way (measured).
-template <int DT, bool PARTIAL, bool CHECKED = false>
-__device__ __forceinline__ void decode_step_raw(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid,
-                                                bool store = true) {
-    if constexpr (DT == SZ_BF16) raw_step_outlined<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
-    else raw_step_body<DT, PARTIAL, CHECKED>(f, hs, dst, valid, store);
+// A raw step inside the coded loop of the contiguous kernels: a call in the
+// BF16 kernel and inline in the E5M2 one, which leaves each one's coded path
+// fastest (measured).
+template <int DT, bool PARTIAL>
+__device__ __forceinline__ void decode_step_raw(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid) {
+    if constexpr (DT == SZ_BF16) raw_step_outlined<DT, PARTIAL>(f, hs, dst, valid);
+    else raw_step_body<DT, PARTIAL, false>(f, hs, dst, valid, true);
 }
 
 // This lane's high bits of step `it` of a raw block within the block's escape
@@ -464,6 +463,34 @@ __device__ __forceinline__ uint32_t load_escape_reg(const uint8_t *comp, const W
     const uint32_t lane = threadIdx.x & 31;
     const uint32_t cnt = b.hi >= b.lo ? b.hi - b.lo : 0u;
     return (lane < cnt && b.hi <= ws.E) ? uint32_t(comp[ws.esc + b.lo + lane]) : 0u;
+}
+
+// Decode raw block blk of tensor t (the warp, from global memory): codes and
+// planes as read_partial gives them, high bits from the block's escape section
+// esc_g.  The paged kernels run it after the block's coded pass, over that
+// pass's output: their coded loop is then the same as without raw blocks,
+// which keeps it fastest (measured).
+template <int DT, int MAXB, bool PAGED>
+__device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
+                                              const uint8_t *esc_g) {
+    using G = DGeo<DT, PAGED>;
+    constexpr int EB = Dt<DT>::kElemBytes;
+    const int lane = threadIdx.x & 31;
+    for (int it = 0; it < G::IT; ++it) {
+        const int64_t e = int64_t(blk) * kBlock + int64_t(it) * 32 * G::LE + int64_t(lane) * G::LE;
+        const int64_t left = int64_t(ws.n) - e;
+        const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
+        if (valid == 0) continue;
+        const DFrag f = read_partial<DT>(p.comp[t], ws, blk, it, valid);
+        uint8_t *dst = p.out[t] + uint64_t(e) * EB;
+        bool store = true;
+        if constexpr (PAGED) {
+            const uint64_t off = elem_offset<EB>(p.pg[t], uint64_t(e));
+            store = off != kBadOffset;  // reported by the coded pass
+            dst = p.out[t] + off;
+        }
+        raw_step_body<DT, true, PAGED>(f, raw_high<DT>(esc_g, it), dst, valid, store);
+    }
 }
 
 template <int MAXB>
@@ -644,18 +671,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                             const bool store = off != kBadOffset;
                             uint8_t *out_q = p.out[t] + off + uint64_t(lane) * G::LE * EB;
                             if (!store && lane == 0) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
-                            if (raw) {
-                                for (int it = 0; it < G::QIT; ++it)
-                                    decode_step_raw<DT, false, true>(read_stage<DT, G>(st_addr, it),
-                                                                     raw_high<DT>(esc_g, q * G::QIT + it),
-                                                                     out_q + it * 512, G::LE, store);
-                            } else {
 #pragma unroll
-                                for (int it = 0; it < G::QIT; ++it) {
-                                    const DFrag f = read_stage<DT, G>(st_addr, it);
-                                    decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE,
-                                                                 running, esc_reg, esc_g, cnt, bad, store);
-                                }
+                            for (int it = 0; it < G::QIT; ++it) {
+                                const DFrag f = read_stage<DT, G>(st_addr, it);
+                                decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE, running,
+                                                             esc_reg, esc_g, cnt, bad, store);
                             }
                         } else if (raw) {
                             for (int it = 0; it < G::QIT; ++it)
@@ -685,11 +705,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                                     dst = p.out[t] + off;
                                     if (!store) set_error(p.ctl, SZ_ERR_INVALID_ARG, p.block_begin[t] + blk);
                                 }
-                                if (raw)
-                                    decode_step_raw<DT, true, true>(f, raw_high<DT>(esc_g, it), dst, valid, store);
-                                else
-                                    decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg,
-                                                                esc_g, cnt, bad, store);
+                                decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg, esc_g,
+                                                            cnt, bad, store);
                             } else if (raw) {
                                 decode_step_raw<DT, true>(f, raw_high<DT>(esc_g, it), out + it * 512, valid);
                             } else {
@@ -700,6 +717,15 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                     }
                 }
                 __syncwarp();  // the stage just read may be refilled from here on
+            }
+            if constexpr (PAGED) {
+                if (raw && !timed_out) {
+                    // A raw block.  The coded pass above took its low exponent
+                    // nibbles for codes (its escape reads stayed inside the block's
+                    // section); decode it again from its planes and high bits.
+                    decode_raw_block<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
+                    bad = false;
+                }
             }
             if (raw) running = cnt;  // a raw block's high bits fill its count exactly
             if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
