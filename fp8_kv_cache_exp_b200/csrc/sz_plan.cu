@@ -199,21 +199,21 @@ __device__ void count_range_paged(uint32_t col, uint32_t inc, const uint8_t *poo
     }
 }
 
-// Add every column into the global histogram g_hist and clear them.
+// Add every column into the global histogram g_hist and clear them: a warp
+// takes one exponent row at a time, one 16-byte load and store per lane.
 template <int DT, int NT>
 __device__ void flush_columns(uint32_t *s_cols, uint32_t *g_hist) {
     using C = PlanCfg<DT>;
-    constexpr int kRow = NT / 2;
+    constexpr int kRowVecs = NT / 2 / 4;  // 16-byte vectors per exponent row
+    static_assert(kRowVecs == 32, "one vector per lane per row");
+    uint4 *rows = reinterpret_cast<uint4 *>(s_cols);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     __syncthreads();
     for (int e = warp; e < C::kBins; e += NT / 32) {
-        uint32_t sum = 0;
-#pragma unroll
-        for (int c = lane; c < kRow; c += 32) {
-            const uint32_t w = s_cols[e * kRow + c];
-            s_cols[e * kRow + c] = 0;
-            sum += (w & 0xFFFFu) + (w >> 16);
-        }
+        const uint4 w = rows[e * kRowVecs + lane];
+        rows[e * kRowVecs + lane] = make_uint4(0, 0, 0, 0);
+        uint32_t sum = (w.x & 0xFFFFu) + (w.x >> 16) + (w.y & 0xFFFFu) + (w.y >> 16) + (w.z & 0xFFFFu) +
+                       (w.z >> 16) + (w.w & 0xFFFFu) + (w.w >> 16);
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0 && sum) atomicAdd(g_hist + e, sum);
     }
@@ -248,36 +248,69 @@ __device__ inline void make_plan_words(uint32_t *s_words, int dtype, uint64_t n,
     s_words[12] = s_words[13] = s_words[14] = s_words[15] = 0;
 }
 
+// Shared scratch of the codebook selection.
+template <int DT>
+struct SelectSmem {
+    uint32_t cnt[Dt<DT>::kBins];   // the tensor's histogram
+    uint32_t list_cnt[Dt<DT>::kBins];  // its non-zero bins, in no particular order
+    uint8_t list_val[Dt<DT>::kBins];
+    uint32_t nnz, sum;
+    uint8_t cb[16];
+    uint32_t words[16];
+};
+
 // Rank every exponent value by (count desc, value asc); write the plan of a
-// tensor of n elements; leave its histogram and ticket zeroed for reuse.
+// tensor of n elements; leave its histogram and ticket zeroed for reuse.  A
+// value's rank counts the values ahead of it in that order; only the non-zero
+// bins are compared (a zero bin comes after all of them, and among zero bins
+// the smaller value first), so the work follows the number of distinct
+// exponents, not the 256 possible ones.
 template <int DT, int NT>
-__device__ void select_codebook(uint32_t *g_hist, uint32_t *g_ticket, uint64_t n, uint8_t *plan,
-                                uint32_t *ctl, uint32_t *s_cnt, uint8_t *s_cb, uint32_t *s_words) {
+__device__ void select_codebook(uint32_t *g_hist, uint32_t *g_ticket, uint64_t n, uint8_t *plan, uint32_t *ctl,
+                                SelectSmem<DT> &S) {
     using C = PlanCfg<DT>;
-    const int tid = threadIdx.x;
-    for (int v = tid; v < C::kBins; v += NT) s_cnt[v] = __ldcg(g_hist + v);
+    static_assert(C::kBins <= NT, "one bin per thread");
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid == 0) S.nnz = S.sum = 0;
     __syncthreads();
-    for (int v = tid; v < C::kBins; v += NT) {
-        const uint32_t cv = s_cnt[v];
-        uint32_t rank = 0;
-#pragma unroll 8
-        for (int u = 0; u < C::kBins; ++u) {
-            const uint32_t cu = s_cnt[u];
-            rank += (cu > cv) | ((cu == cv) & (u < v));
+    const uint32_t c = tid < C::kBins ? __ldcg(g_hist + tid) : 0u;
+    if (tid < C::kBins) {
+        S.cnt[tid] = c;
+        if (c) {
+            const uint32_t pos = atomicAdd(&S.nnz, 1u);
+            S.list_cnt[pos] = c;
+            S.list_val[pos] = uint8_t(tid);
         }
-        if (rank < kCodes) s_cb[rank] = uint8_t(v);
+    }
+    const uint32_t wsum = __reduce_add_sync(0xffffffffu, c);  // n < 2^32: no overflow
+    if (lane == 0 && wsum) atomicAdd(&S.sum, wsum);
+    __syncthreads();
+    if (tid < C::kBins) {
+        const uint32_t nnz = S.nnz, v = uint32_t(tid);
+        uint32_t rank = kCodes;
+        if (c) {
+            rank = 0;
+            for (uint32_t j = 0; j < nnz; ++j) {
+                const uint32_t cu = S.list_cnt[j], u = S.list_val[j];
+                rank += (cu > c) | ((cu == c) & (u < v));
+            }
+        } else if (nnz < kCodes) {
+            uint32_t below = 0;  // non-zero bins of smaller value
+            for (uint32_t j = 0; j < nnz; ++j) below += S.list_val[j] < v;
+            rank = nnz + (v - below);
+        }
+        if (rank < kCodes) S.cb[rank] = uint8_t(v);
     }
     __syncthreads();
     if (tid == 0) {
-        uint64_t sum = 0, covered = 0;
-        for (int v = 0; v < C::kBins; ++v) sum += s_cnt[v];
-        for (int c = 0; c < int(kCodes); ++c) covered += s_cnt[s_cb[c]];
-        if (sum != n) set_error(ctl, SZ_ERR_INTERNAL, 1);
-        make_plan_words(s_words, DT, n, n - covered, s_cb);
+        uint64_t covered = 0;
+        for (int k = 0; k < int(kCodes); ++k) covered += S.cnt[S.cb[k]];
+        if (S.sum != n) set_error(ctl, SZ_ERR_INTERNAL, 1);
+        make_plan_words(S.words, DT, n, n - covered, S.cb);
     }
     __syncthreads();
-    store_plan(plan, s_words);
-    for (int v = tid; v < C::kBins; v += NT) g_hist[v] = 0;
+    store_plan(plan, S.words);
+    if (tid < C::kBins) g_hist[tid] = 0;
     if (tid == 0) *g_ticket = 0;
 }
 
@@ -286,9 +319,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
     using C = PlanCfg<DT>;
     extern __shared__ uint32_t s_cols[];  // C::kBins * NT/2 words of two 16-bit counters, then page ids
     int32_t *s_ids = reinterpret_cast<int32_t *>(s_cols + C::kBins * (NT / 2));
-    __shared__ uint32_t s_cnt[C::kBins];
-    __shared__ uint8_t s_cb[16];
-    __shared__ uint32_t s_words[16];
+    __shared__ SelectSmem<DT> s_sel;
     __shared__ uint32_t s_last;
     const int tid = threadIdx.x;
     const uint32_t col = smem_u32(s_cols + (tid % (NT / 2)));
@@ -301,10 +332,10 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
             if (tid == 0) {
                 uint8_t cb[kCodes];
                 for (int c = 0; c < int(kCodes); ++c) cb[c] = uint8_t(c);
-                make_plan_words(s_words, DT, 0, 0, cb);
+                make_plan_words(s_sel.words, DT, 0, 0, cb);
             }
             __syncthreads();
-            store_plan(p.plans + 64 * size_t(t), s_words);
+            store_plan(p.plans + 64 * size_t(t), s_sel.words);
             __syncthreads();
         }
     }
@@ -312,7 +343,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
     const uint64_t lo = p.total_items * blockIdx.x / gridDim.x;
     const uint64_t hi = p.total_items * (blockIdx.x + 1) / gridDim.x;
     if (lo >= hi) return;
-    for (int i = tid; i < C::kBins * (NT / 2); i += NT) s_cols[i] = 0;
+    for (int i = tid; i < C::kBins * (NT / 2) / 4; i += NT) reinterpret_cast<uint4 *>(s_cols)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
 
     int t = find_tensor<uint64_t, MAXB>(p.item_begin, p.T, lo);
@@ -352,8 +383,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
         }
         __syncthreads();
         if (s_last) {
-            select_codebook<DT, NT>(g_hist, p.ticket + t, p.n[t], p.plans + 64 * size_t(t), p.ctl,
-                                    s_cnt, s_cb, s_words);
+            select_codebook<DT, NT>(g_hist, p.ticket + t, p.n[t], p.plans + 64 * size_t(t), p.ctl, s_sel);
             __syncthreads();
         }
         i = i_end;
