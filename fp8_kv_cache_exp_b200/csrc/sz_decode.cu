@@ -471,8 +471,8 @@ __device__ __forceinline__ uint32_t load_escape_reg(const uint8_t *comp, const W
 // pass's output: their coded loop is then the same as without raw blocks,
 // which keeps it fastest (measured).
 template <int DT, int MAXB, bool PAGED>
-__device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
-                                              const uint8_t *esc_g) {
+__device__ __forceinline__ void raw_block_body(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
+                                               const uint8_t *esc_g) {
     using G = DGeo<DT, PAGED>;
     constexpr int EB = Dt<DT>::kElemBytes;
     const int lane = threadIdx.x & 31;
@@ -491,6 +491,20 @@ __device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, in
         }
         raw_step_body<DT, true, PAGED>(f, raw_high<DT>(esc_g, it), dst, valid, store);
     }
+}
+
+template <int DT, int MAXB, bool PAGED>
+__device__ __noinline__ void raw_block_outlined(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
+                                                const uint8_t *esc_g) {
+    raw_block_body<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
+}
+
+// A call in the BF16 kernel, inline in the E5M2 one (each the faster, measured).
+template <int DT, int MAXB, bool PAGED>
+__device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
+                                                 const uint8_t *esc_g) {
+    if constexpr (DT == SZ_BF16) raw_block_outlined<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
+    else raw_block_body<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
 }
 
 template <int MAXB>
