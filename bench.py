@@ -98,16 +98,24 @@ def load_peaks():
 KERNEL_SOURCES = ("sz_common.cuh", "sz_plan.cu", "sz_encode.cu", "sz_decode.cu")
 
 
+def _code_only(src: str) -> str:
+    """C/CUDA source without comments and blank lines (comments do not change a kernel)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    lines = [re.sub(r"//.*", "", ln).rstrip() for ln in src.splitlines()]
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the device-code sources (which kernels a profile describes); host-only
-    files (the C-ABI layer, the header) do not change it."""
+    """Hash of the device-code sources, comments left out (which kernels a profile
+    describes); host-only files (the C-ABI layer, the header) do not change it."""
     import hashlib
     files = [os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", f) for f in KERNEL_SOURCES]
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

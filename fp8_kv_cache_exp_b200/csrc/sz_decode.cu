@@ -23,7 +23,11 @@
 //     two) and the escape bytes from a shuffle -- an E5M2 lane's single escape
 //     enters through its table's code-15 byte; the elements are reassembled
 //     with byte permutes and integer multiply-adds and written with 16-byte
-//     stores (512 contiguous bytes per warp instruction).
+//     stores (512 contiguous bytes per warp instruction);
+//   - a raw block (header flag set and an offsets-table count equal to the
+//     block's raw size) is rebuilt from its low exponent nibbles and the high
+//     bits in its escape section: step by step in the contiguous kernels, in a
+//     pass after the block's coded pass in the paged ones.
 #include <type_traits>
 
 #include "sz_common.cuh"

@@ -21,7 +21,11 @@
 //   4. the chunk's offsets-table entries and escapes are written contiguously
 //      (a chunk whose escapes overflow the stage re-codes its input and writes
 //      them directly); the tensor's last chunk writes the header, offsets[nb]
-//      and the zero padding.
+//      and the zero padding;
+//   5. with raw blocks allowed (header flag), a block whose escapes reach its
+//      raw size is stored raw: its chunk re-reads the input, writes the low
+//      exponent nibbles over the codes and the high bits to the escape
+//      section, and the last chunk writes the exact E and total.
 #include <type_traits>
 
 #include "sz_common.cuh"
