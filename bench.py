@@ -396,7 +396,9 @@ def run_ours(args, rank, world, device):
     value = raw_all / (ms_step * 1e-3) / 1e9
 
     peak, peak_kind = load_peaks()
-    launches_per_step = (2 if args.reuse else 3) * len(groups)
+    # plan, encode, decode per call (no plan with --reuse); paged and E5M2 decode add their
+    # raw-block pass
+    launches_per_step = ((2 if args.reuse else 3) + (1 if args.paged or dt == 1 else 0)) * len(groups)
     kern = {
         "plan": {"ms": t_plan, "bytes": wl.raw_bytes + 64 * T},
         "encode": {"ms": t_enc, "bytes": wl.raw_bytes + stream_bytes},

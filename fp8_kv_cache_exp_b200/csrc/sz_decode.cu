@@ -26,8 +26,8 @@
 //     stores (512 contiguous bytes per warp instruction);
 //   - a raw block (header flag set and an offsets-table count equal to the
 //     block's raw size) is rebuilt from its low exponent nibbles and the high
-//     bits in its escape section: step by step in the contiguous kernels, in a
-//     pass after the block's coded pass in the paged ones.
+//     bits in its escape section: step by step in the contiguous BF16 kernel,
+//     and by a second kernel (raw_pass_kernel) after the others.
 #include <type_traits>
 
 #include "sz_common.cuh"
@@ -427,9 +427,8 @@ __device__ __noinline__ void raw_step_outlined(const DFrag &f, const uint8_t *hs
     raw_step_body<DT, PARTIAL, false>(f, hs, dst, valid, true);
 }
 
-// A raw step inside the coded loop of the contiguous kernels: a call in the
-// BF16 kernel and inline in the E5M2 one, which leaves each one's coded path
-// fastest (measured).
+// A raw step inside the coded loop of the contiguous BF16 kernel, as a call:
+// that leaves its coded path fastest (measured).
 template <int DT, bool PARTIAL>
 __device__ __forceinline__ void decode_step_raw(const DFrag &f, const uint8_t *hs, uint8_t *dst, int valid) {
     if constexpr (DT == SZ_BF16) raw_step_outlined<DT, PARTIAL>(f, hs, dst, valid);
@@ -471,12 +470,11 @@ __device__ __forceinline__ uint32_t load_escape_reg(const uint8_t *comp, const W
 
 // Decode raw block blk of tensor t (the warp, from global memory): codes and
 // planes as read_partial gives them, high bits from the block's escape section
-// esc_g.  The paged kernels run it after the block's coded pass, over that
-// pass's output: their coded loop is then the same as without raw blocks,
-// which keeps it fastest (measured).
+// esc_g.  Used by raw_pass_kernel, over what the decode kernel's coded pass
+// wrote.
 template <int DT, int MAXB, bool PAGED>
-__device__ __forceinline__ void raw_block_body(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
-                                               const uint8_t *esc_g) {
+__device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
+                                                 const uint8_t *esc_g) {
     using G = DGeo<DT, PAGED>;
     constexpr int EB = Dt<DT>::kElemBytes;
     const int lane = threadIdx.x & 31;
@@ -495,20 +493,6 @@ __device__ __forceinline__ void raw_block_body(const DecodeParams<MAXB> &p, int 
         }
         raw_step_body<DT, true, PAGED>(f, raw_high<DT>(esc_g, it), dst, valid, store);
     }
-}
-
-template <int DT, int MAXB, bool PAGED>
-__device__ __noinline__ void raw_block_outlined(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
-                                                const uint8_t *esc_g) {
-    raw_block_body<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
-}
-
-// A call in the BF16 kernel, inline in the E5M2 one (each the faster, measured).
-template <int DT, int MAXB, bool PAGED>
-__device__ __forceinline__ void decode_raw_block(const DecodeParams<MAXB> &p, int t, const WarpStream &ws, uint32_t blk,
-                                                 const uint8_t *esc_g) {
-    if constexpr (DT == SZ_BF16) raw_block_outlined<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
-    else raw_block_body<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
 }
 
 template <int MAXB>
@@ -695,7 +679,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                                 decode_step<DT, false, true>(f, tab_addr, ws.xt, out_q + it * 512, G::LE, running,
                                                              esc_reg, esc_g, cnt, bad, store);
                             }
-                        } else if (raw) {
+                        } else if (DT == SZ_BF16 && raw) {
                             for (int it = 0; it < G::QIT; ++it)
                                 decode_step_raw<DT, false>(read_stage<DT, G>(st_addr, it),
                                                            raw_high<DT>(esc_g, q * G::QIT + it),
@@ -725,7 +709,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                                 }
                                 decode_step<DT, true, true>(f, tab_addr, ws.xt, dst, valid, running, esc_reg, esc_g,
                                                             cnt, bad, store);
-                            } else if (raw) {
+                            } else if (DT == SZ_BF16 && raw) {
                                 decode_step_raw<DT, true>(f, raw_high<DT>(esc_g, it), out + it * 512, valid);
                             } else {
                                 decode_step<DT, true>(f, tab_addr, ws.xt, out + it * 512, valid, running, esc_reg,
@@ -736,14 +720,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                 }
                 __syncwarp();  // the stage just read may be refilled from here on
             }
-            if constexpr (PAGED) {
-                if (raw && !timed_out) {
-                    // A raw block.  The coded pass above took its low exponent
-                    // nibbles for codes (its escape reads stayed inside the block's
-                    // section); decode it again from its planes and high bits.
-                    decode_raw_block<DT, MAXB, PAGED>(p, t, ws, blk, esc_g);
-                    bad = false;
-                }
+            if constexpr (PAGED || DT == SZ_FP8_E5M2) {
+                // A raw block.  The coded pass above took its low exponent nibbles
+                // for codes (its escape reads stayed inside the block's section);
+                // raw_pass_kernel, launched next, decodes it from its planes and
+                // high bits.
+                if (raw) bad = false;
             }
             if (raw) running = cnt;  // a raw block's high bits fill its count exactly
             if (ok && !timed_out) bad = __any_sync(0xffffffffu, bad) || running != cnt;
@@ -794,6 +776,43 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel_paged(const __grid_consta
     decode_body<DT, MAXB, true>(p);
 }
 
+// Second pass of the paged kernels and of the E5M2 one: one CTA per tensor
+// re-reads the stream's header and, if it allows raw blocks, decodes each raw
+// block from its planes and high bits over what the coded pass wrote.  A
+// stream without the flag costs one header read.  Keeping raw blocks out of
+// those kernels' loops keeps the loops as fast as without them (measured).
+template <int DT, int MAXB, bool PAGED>
+__global__ void __launch_bounds__(NT) raw_pass_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
+    __shared__ uint32_t s_tab[NW][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = int(blockIdx.x);
+    if (t >= p.T || p.n[t] == 0) return;
+    WarpStream ws;
+    warp_open_stream<DT, MAXB>(p, t, s_tab[warp], ws);  // each warp, for its own copy of ws
+    if (!ws.ok || !ws.raw_ok) return;
+    const uint8_t *comp = p.comp[t];
+    const uint32_t *tabw = reinterpret_cast<const uint32_t *>(comp + 64);
+    for (uint32_t b0 = uint32_t(warp) * 32; b0 < ws.nb; b0 += NW * 32) {
+        const uint32_t b = b0 + uint32_t(lane);
+        bool raw = false;
+        uint32_t lo = 0;
+        if (b < ws.nb) {
+            lo = tabw[b];
+            const uint32_t hi = tabw[b + 1];
+            const uint64_t first = uint64_t(b) * kBlock;
+            const uint32_t m = uint32_t(min(uint64_t(kBlock), ws.n - first));
+            raw = lo <= hi && hi <= ws.E && hi - lo == raw_block_bytes<DT>(m);
+        }
+        uint32_t mask = __ballot_sync(0xffffffffu, raw);
+        while (mask) {
+            const int l = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const uint32_t blo = __shfl_sync(0xffffffffu, lo, l);
+            decode_raw_block<DT, MAXB, PAGED>(p, t, ws, b0 + uint32_t(l), comp + ws.esc + blo);
+        }
+    }
+}
+
 template <int DT, int MAXB, bool PAGED>
 sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     auto kern = PAGED ? decode_kernel_paged<DT, MAXB> : decode_kernel<DT, MAXB>;
@@ -821,6 +840,7 @@ sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     const uint64_t need = cdiv(p.total_blocks, NW);
     const uint64_t grid = need < resident ? need : resident;
     kern<<<unsigned(grid), NT, smem, stream>>>(p);
+    if (PAGED || DT == SZ_FP8_E5M2) raw_pass_kernel<DT, MAXB, PAGED><<<unsigned(a.T), NT, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
 
