@@ -229,3 +229,26 @@ def test_uniform_bits_full_size():
     raw = uniform(rng, n, 0)
     ref = check(0, raw)
     assert ref.size <= raw.size + fieldcodec.align256(64 + 4 * (n // 4096 + 1)) + 512
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_corrupt_raw_stream_is_reported(dtype):
+    """A flagged stream whose offsets table no longer marks its raw blocks is
+    reported as corrupt (the decode stays inside the stream and the output)."""
+    m = sz()
+    rng = np.random.default_rng(71 + dtype)
+    n = 3 * 4096 + 100
+    raw = uniform(rng, n, dtype)
+    st, _, stream = gpu_encode_raw(dtype, raw)
+    assert st == 0
+    for what in ("count_plus_one", "flag_cleared"):
+        bad = stream.copy()
+        if what == "count_plus_one":
+            bad[68] ^= 1  # offsets[1]: block 0's count is no longer its raw size
+        else:
+            bad[39] = 0   # without the flag the raw blocks read as coded ones
+        comp = torch.from_numpy(bad).cuda()
+        out = torch.empty(n * es(dtype), dtype=torch.uint8, device="cuda")
+        ws = m.new_workspace(dtype, [n])
+        m.sz_decode(dtype, comp, out, ws)
+        assert m.sz_last_device_status(ws) == m.SZ_ERR_CORRUPT_STREAM, what

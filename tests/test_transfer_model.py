@@ -25,3 +25,4 @@ def test_pipeline_model_by_hand():
     # uneven layers
     assert pipelined_seconds([(1, 1, 1), (3, 1, 1)]) == 6   # layer 1: 4, 5, 6
     assert pipelined_seconds([]) == 0.0
+
