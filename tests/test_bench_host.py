@@ -9,3 +9,23 @@ def test_kernel_hash_ignores_comments():
     c = "int f(int x) {\n    return 3 * x;\n}\n"
     assert bench._code_only(a) == bench._code_only(b)
     assert bench._code_only(a) != bench._code_only(c)
+
+
+def test_reference_arm_line_on_cpu():
+    """`bench.py --impl reference` times the CPU oracle and prints the contract's JSON line:
+    the same metric and unit, an e2e object with no host-device bytes, and a cpu_baseline
+    of kind "oracle" (it needs no GPU)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    import bench
+    assert line["metric"] == bench.METRIC
