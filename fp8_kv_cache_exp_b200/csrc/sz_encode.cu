@@ -585,14 +585,22 @@ __device__ __forceinline__ void warp_load_plan(const EncodeParams<MAXB> &p, int 
     __syncwarp();
     const Header H = load_header(reinterpret_cast<const uint8_t *>(W.hdr));
     const uint32_t lut = lut_addr(W);
-    for (int x = lane; x < 256; x += 32) {
-        // BF16: x is the exponent; E5M2: x is the element byte
-        const uint32_t e = (DT == SZ_BF16) ? uint32_t(x) : (uint32_t(x) >> 2) & 0x1Fu;
-        uint32_t code = kEscape;
+    // every entry escapes (8 bytes per lane) ...
+    sts_u64(lut + uint32_t(lane) * 8u, 0x0F0F0F0F0F0F0F0Full);
+    __syncwarp();
+    // ... except those of the codebook's values: lane c writes code c.  A value
+    // outside the exponent range writes nothing (plan_ok then rejects the plan).
+    if (lane < int(kCodes)) {
+        const uint32_t e = cb_byte(H.cbw, lane);
+        if (e < uint32_t(Dt<DT>::kBins)) {
+            if constexpr (DT == SZ_BF16) {
+                sts_u8(lut + e, uint32_t(lane));  // BF16 entries are indexed by the exponent
+            } else {
 #pragma unroll
-        for (int c = 0; c < int(kCodes); ++c)
-            if (cb_byte(H.cbw, c) == e) code = uint32_t(c);
-        sts_u8(lut + uint32_t(x), code);
+                for (uint32_t sm = 0; sm < 8; ++sm)  // E5M2 entries by the element byte: sign, mantissa
+                    sts_u8(lut + ((sm >> 2) << 7 | e << 2 | (sm & 3u)), uint32_t(lane));
+            }
+        }
     }
     __syncwarp();
 }
