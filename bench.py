@@ -106,11 +106,19 @@ def _code_only(src: str) -> str:
     return "\n".join(ln for ln in lines if ln.strip())
 
 
-def kernel_source_hash() -> str:
-    """Hash of the device-code sources, comments left out (which kernels a profile
-    describes); host-only files (the C-ABI layer, the header) do not change it."""
+# the sources each kernel's code comes from
+KERNEL_FILES = {"plan_kernel": ("sz_common.cuh", "sz_plan.cu"),
+                "encode_kernel": ("sz_common.cuh", "sz_encode.cu"),
+                "decode_kernel": ("sz_common.cuh", "sz_decode.cu")}
+
+
+def kernel_source_hash(kernel: str = None) -> str:
+    """Hash of the device-code sources, comments left out: of all of them (which build
+    a profile describes), or of one kernel's (whether its recorded traffic still
+    applies).  Host-only files (the C-ABI layer, the header) do not change it."""
     import hashlib
-    files = [os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", f) for f in KERNEL_SOURCES]
+    names = KERNEL_SOURCES if kernel is None else KERNEL_FILES[kernel]
+    files = [os.path.join(ROOT, "fp8_kv_cache_exp_b200", "csrc", f) for f in names]
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())
@@ -126,7 +134,7 @@ def profiled_traffic(kernel: str, workload: str):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for line in lines:
         parts = line.split()
         if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
