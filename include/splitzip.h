@@ -266,8 +266,8 @@ sz_status sz_encode_reuse_paged_batched(sz_dtype dtype, int T, const sz_plan_t *
  * directly (peer access over NVLink).  After it, sz_decode* on `device` may be
  * given streams that live on `peer`: the decode kernel then pulls each
  * stream's bytes across the link itself, with the same 1-D bulk copies it uses
- * for local streams (no multicast), so the transfer overlaps the decoding
- * tile by tile and the stream never lands in `device`'s memory.
+ * for local streams (each CTA fetches its own tiles), so the transfer overlaps
+ * the decoding tile by tile and the stream never lands in `device`'s memory.
  * SZ_OK if access is enabled (or already was; device == peer needs nothing),
  * SZ_ERR_CUDA if the two devices cannot reach each other. */
 sz_status sz_enable_peer_access(int device, int peer);
