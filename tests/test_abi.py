@@ -87,3 +87,16 @@ def test_plan_set_flags_host_checks(lib):
     assert f(1, None, 1, None) == 1
     assert f(1, fake + 4, 1, None) == 1
     assert f(1, fake, 2, None) == 1
+
+
+def test_binding_host_checks():
+    """The binding's own argument checks on a batch (no GPU call is reached)."""
+    import torch
+    import fp8_kv_cache_exp_b200 as sz
+    plans = torch.zeros((2, 64), dtype=torch.uint8)
+    xs = [torch.zeros(16, dtype=torch.bfloat16)]
+    with pytest.raises(ValueError):
+        sz.Batch(sz.SZ_BF16, xs, [], torch.zeros(1024, dtype=torch.uint8), plans)
+    with pytest.raises(ValueError):
+        sz.Batch(sz.SZ_BF16, None, [torch.zeros(256, dtype=torch.uint8)], torch.zeros(1024, dtype=torch.uint8),
+                 plans, src_pages=[object()])
