@@ -99,4 +99,4 @@ def test_binding_host_checks():
         sz.Batch(sz.SZ_BF16, xs, [], torch.zeros(1024, dtype=torch.uint8), plans)
     with pytest.raises(ValueError):
         sz.Batch(sz.SZ_BF16, None, [torch.zeros(256, dtype=torch.uint8)], torch.zeros(1024, dtype=torch.uint8),
-                 plans, src_pages=[object()])
+                 plans, src_pages=[sz.sz_paged_t()])  # paged without element counts
