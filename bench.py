@@ -12,7 +12,14 @@ round trip (plan + encode + decode); encode (plan + encode) and decode rates,
 per-kernel roofline fractions and the compression ratio ride along.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload llama3-8b|qwen3-32b-layer|...] [--mode batch|per_layer]
+                  [--workload llama3-8b|qwen3-32b-layer|qwen3-30b-a3b-e5m2|stress-uniform-bf16]
+                  [--mode batch|per_layer] [--reuse] [--paged TOKENS] [--raw-blocks]
+                  [--transfer] [--no-graph] [--no-e2e] [--layers N]
+
+The step is timed with per-kernel CUDA events over direct launches, then captured
+once as a CUDA graph and replayed (`ms_per_step`, `value`).  `e2e` repeats the
+step through the public API from pinned host memory and back, pipelining the
+copies of consecutive steps with the kernels.
 
 `--impl reference` times the CPU oracle (plain single-threaded C) on a bounded
 sample of the same workload: the only reference implementation there is.
