@@ -84,3 +84,22 @@ def test_decode_rejects_wrong_n(orc):
     raw, s = _stream(orc)
     rc, _ = orc.decode_status(s, 9999, 0)
     assert rc == oracle.ERR_ARG
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_decode_rejects_broken_raw_marker(orc, dtype):
+    """A flagged stream whose offsets table no longer marks its raw blocks, or that lost
+    its flag, is rejected (the same cases the GPU decoder reports)."""
+    rng = np.random.default_rng(9 + dtype)
+    n = 3 * 4096 + 100
+    raw = rng.integers(0, 256, n * (2 if dtype == 0 else 1)).astype(np.uint8)
+    s = orc.encode(dtype, raw, raw_blocks=True)
+    assert np.array_equal(orc.decode(s, n, dtype), raw)
+    for what in ("count_plus_one", "flag_cleared"):
+        bad = s.copy()
+        if what == "count_plus_one":
+            bad[68] ^= 1
+        else:
+            bad[39] = 0
+        rc, _ = orc.decode_status(bad, n, dtype)
+        assert rc == oracle.ERR_CORRUPT, what
