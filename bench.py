@@ -9,23 +9,38 @@ flush is needed between steps.
 
 Prints one JSON line.  `value` is raw input bytes per second through a full
 round trip (plan + encode + decode); encode (plan + encode) and decode rates,
-per-kernel roofline fractions and the compression ratio ride along.
+per-kernel roofline fractions and the compression ratio ride along.  With the
+default workload the line also carries `configs`: the other KV workloads,
+measured in the same run --
+
+  qwen3-32b            64 layers x {K,V} x [131072, 8, 128] bf16 (34.4 GB),
+                       generated on the device one layer at a time and coded
+                       layer by layer (537 MB per call), L2 flushed before
+                       each layer;
+  qwen3-30b-a3b-e5m2   48 layers x {K,V} x [32768, 4, 128] FP8 E5M2, one batch;
+  llama3-8b-per-layer  the Llama-3-8B KV coded layer by layer (33.5 MB per
+                       call), 32 calls per step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload llama3-8b|qwen3-32b-layer|qwen3-30b-a3b-e5m2|stress-uniform-bf16]
                   [--mode batch|per_layer] [--reuse] [--paged TOKENS] [--raw-blocks]
-                  [--transfer] [--no-graph] [--no-e2e] [--layers N]
+                  [--transfer] [--no-graph] [--no-e2e] [--no-records] [--layers N]
+                  [--kernel-reps R]
 
-The step is timed with per-kernel CUDA events over direct launches, then captured
-once as a CUDA graph and replayed (`ms_per_step`, `value`).  `e2e` repeats the
-step through the public API from pinned host memory and back, pipelining the
-copies of consecutive steps with the kernels.
+Timing: every figure comes from CUDA events on the launching stream.  The K
+timed steps are the step captured once as a CUDA graph and replayed
+(`ms_per_step`, `value`); `step_stats` adds the median over max(K, 50)
+further replays.  Per-kernel figures come from each kernel's own graph (its
+launches of one step), replayed max(K, R) times in step order: `ms` is the
+mean, `ms_median` the median.  `e2e` repeats the step through the public API
+from pinned host memory and back, pipelining the copies of consecutive steps
+with the kernels.
 
-`--impl reference` times the CPU oracle (plain single-threaded C) on a bounded
-sample of the same workload: the only reference implementation there is.
-For N > 1 (torchrun), every rank codes its own batch of the same size (weak
-scaling: the tensors are independent, no data-path collective); timing is the
-max over ranks.
+`--impl reference` times the CPU oracle (plain single-threaded C, pinned to one
+core) on a bounded sample of the same workload: the only reference
+implementation there is.  For N > 1 (torchrun), every rank codes its own batch
+of the same size (weak scaling: the tensors are independent, no data-path
+collective); timing is the max over ranks.
 """
 import argparse
 import datetime
@@ -207,6 +222,63 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def head_start(ms: float = 2.0):
+    """Keep the GPU busy for about `ms` so that the host enqueues the work that
+    follows before the GPU reaches it (no host gap inside a measurement)."""
+    torch.cuda._sleep(int(ms * 2e6))
+
+
+def capture_graph(fn, stream, device):
+    """fn() (calls that only enqueue kernels) captured once as a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device=device)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap), torch.cuda.graph(g, stream=cap):
+        fn()
+    stream.wait_stream(cap)
+    return g
+
+
+def graph_part_times(parts: dict, reps: int, stream, device, warmup: int = 3) -> dict:
+    """Each of `parts` (name -> fn enqueuing kernels) captured as its own CUDA
+    graph; all of them replayed in order `reps` times with a CUDA event between
+    consecutive graphs.  Returns name -> list of ms per replay."""
+    graphs = {k: capture_graph(fn, stream, device) for k, fn in parts.items()}
+    for _ in range(warmup):
+        for g in graphs.values():
+            g.replay()
+    torch.cuda.synchronize()
+    names = list(graphs)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(reps)]
+    head_start()
+    for r in range(reps):
+        ev[r][0].record(stream)
+        for i, k in enumerate(names):
+            graphs[k].replay()
+            ev[r][i + 1].record(stream)
+    torch.cuda.synchronize()
+    out = {k: [ev[r][i].elapsed_time(ev[r][i + 1]) for r in range(reps)] for i, k in enumerate(names)}
+    del graphs
+    return out
+
+
+def kernel_figures(times_ms, nbytes: int, peak: float) -> dict:
+    """Mean and median of a kernel's times and its algorithmic GB/s and fraction
+    of peak (from the mean)."""
+    ms = sum(times_ms) / len(times_ms)
+    med = statistics.median(times_ms)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "ms_median": med, "gbs": gbs, "frac": gbs / peak,
+            "frac_median": nbytes / (med * 1e-3) / 1e9 / peak}
+
+
+def check_status(sz, workspaces, where: str):
+    for w in workspaces:
+        st = sz.sz_last_device_status(w)
+        if st != 0:
+            raise RuntimeError("device status (%s): %s" % (where, sz.sz_status_string(st)))
+
+
 # ------------------------------------------------------------- our arm
 
 class Workload:
@@ -262,9 +334,10 @@ def paged_pools(wl, page_tokens: int, device):
     return src_pool, dst_pool, src_tabs, dst_tabs, page_elems
 
 
-def run_ours(args, rank, world, device):
+def run_ours(args, rank, world, device, wl=None):
     import fp8_kv_cache_exp_b200 as sz
-    wl = Workload(args.workload, rank, world, device, args.layers)
+    if wl is None:
+        wl = Workload(args.workload, rank, world, device, args.layers)
     if wl.cfg is None and (args.mode != "batch" or args.paged or args.transfer or args.layers):
         raise SystemExit("the stress workload is one flat tensor: batch mode only")
     dt = wl.dtype
@@ -339,72 +412,61 @@ def run_ours(args, rank, world, device):
 
     for _ in range(args.warmup):
         plan_all(); encode_all(); decode_all()
+    torch.cuda.synchronize()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    R = max(K, args.kernel_reps)
+    # Per-kernel figures: each kernel's launches of one step captured as a graph
+    # of its own (no host gap inside a measurement), replayed in step order.
+    parts = {"encode": encode_all, "decode": decode_all}
+    if not args.reuse:
+        parts = {"plan": plan_all, **parts}
+    kt = graph_part_times(parts, R, stream, device, args.warmup)
+    check_status(sz, ws_g, "kernel timing")
+
+    # The timed region: K steps, the whole step captured once as a CUDA graph
+    # (--no-graph: direct launches), bracketed by a barrier and a synchronize.
+    graph = None
+    if args.graph:
+        graph = capture_graph(lambda: (plan_all(), encode_all(), decode_all()), stream, device)
+        for _ in range(args.warmup):
+            graph.replay()
+    step = graph.replay if graph is not None else (lambda: (plan_all(), encode_all(), decode_all()))
     clocks = ClockSampler(gpu_uuid(device))
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    start = torch.cuda.Event(enable_timing=True)
-    stop = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    head_start()
+    ev[0].record(stream)
     for k in range(K):
-        ev[k][0].record(stream)
-        plan_all()
-        ev[k][1].record(stream)
-        encode_all()
-        ev[k][2].record(stream)
-        decode_all()
-        ev[k][3].record(stream)
-    stop.record(stream)
+        step()
+        ev[k + 1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    total_ms = start.elapsed_time(stop)
-    t_plan = sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K
-    t_enc = sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K
-    t_dec = sum(ev[k][2].elapsed_time(ev[k][3]) for k in range(K)) / K
-    for w in ws_g:
-        st = sz.sz_last_device_status(w)
-        if st != 0:
-            raise RuntimeError("device status after timing: %s" % sz.sz_status_string(st))
-    if args.graph:
-        # The same step captured once as a CUDA graph and replayed: the calls
-        # launch kernels only (no allocation, no synchronisation), so they capture
-        # as they are; replay removes the host launch gaps between the calls.
-        graph = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(device=device)
-        cap.wait_stream(stream)
-        with torch.cuda.stream(cap), torch.cuda.graph(graph, stream=cap):
-            plan_all(); encode_all(); decode_all()
-        stream.wait_stream(cap)
-        for _ in range(args.warmup):
-            graph.replay()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for _ in range(K):
-            graph.replay()
-        g1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        total_ms = g0.elapsed_time(g1)
-        for w in ws_g:
-            st = sz.sz_last_device_status(w)
-            if st != 0:
-                raise RuntimeError("device status after graph replay: %s" % sz.sz_status_string(st))
-        if not args.paged:
-            for x, d in zip(wl.xs, decs):
-                if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
-                    raise RuntimeError("round trip mismatch after graph replay")
-        del graph
+    total_ms = ev[0].elapsed_time(ev[K])
+    step_ms = [ev[k].elapsed_time(ev[k + 1]) for k in range(K)]
+    check_status(sz, ws_g, "timed steps")
+    # the median step over more replays (outside the timed region)
+    reps = max(K, 50)
+    ev2 = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    head_start()
+    ev2[0].record(stream)
+    for k in range(reps):
+        step()
+        ev2[k + 1].record(stream)
+    torch.cuda.synchronize()
+    more = sorted(ev2[k].elapsed_time(ev2[k + 1]) for k in range(reps))
+    check_status(sz, ws_g, "step replays")
+    if not args.paged:
+        for x, d in zip(wl.xs, decs):
+            if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
+                raise RuntimeError("round trip mismatch after timing")
+    del graph
 
     ms_step = max_over_ranks(total_ms / K, world, device)
     raw_all = sum_over_ranks(float(wl.raw_bytes), world, device)
@@ -414,29 +476,26 @@ def run_ours(args, rank, world, device):
     # plan, encode, decode per call (no plan with --reuse); paged and E5M2 decode add their
     # raw-block pass
     launches_per_step = ((2 if args.reuse else 3) + (1 if args.paged or dt == 1 else 0)) * len(groups)
-    kern = {
-        "plan": {"ms": t_plan, "bytes": wl.raw_bytes + 64 * T},
-        "encode": {"ms": t_enc, "bytes": wl.raw_bytes + stream_bytes},
-        "decode": {"ms": t_dec, "bytes": stream_bytes + wl.raw_bytes},
-    }
-    if args.reuse:
-        del kern["plan"]
-    for k in kern.values():
-        k["gbs"] = k["bytes"] / (k["ms"] * 1e-3) / 1e9
-        k["frac"] = k["gbs"] / peak
+    kbytes = {"plan": wl.raw_bytes + 64 * T, "encode": wl.raw_bytes + stream_bytes,
+              "decode": stream_bytes + wl.raw_bytes}
+    kern = {k: kernel_figures(kt[k], kbytes[k], peak) for k in kt}
     dom = max(kern, key=lambda k: kern[k]["ms"])
     key = wl.name + ("+paged%d" % args.paged if args.paged else "")
-    traffic = profiled_traffic(dom + "_kernel", key) if world == 1 and not args.layers else None
+    traffic = profiled_traffic(dom + "_kernel", key) if world == 1 and not args.layers and \
+        args.mode == "batch" else None
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(kern[dom]["gbs"], 1), "peak": peak,
             "unit": "GB/s", "frac": round(kern[dom]["frac"], 4),
-            "traffic": traffic, "algorithmic_bytes": kern[dom]["bytes"],
-            "peak_source": peak_kind}
+            "traffic": traffic, "algorithmic_bytes": kbytes[dom],
+            "peak_source": peak_kind, "launches_timed": R,
+            "timing": "mean of %d replays of the kernel's own graph (one step's launches)" % R}
+    t_plan = kern["plan"]["ms"] if "plan" in kern else 0.0
+    t_enc, t_dec = kern["encode"]["ms"], kern["decode"]["ms"]
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "u8" if dt == 1 else "u16", "data": "synthetic (seeded generator, see DESIGN.md)",
+        "dtype": "u8" if dt == 1 else "u16", "data": "synthetic (seeded generator: kvgen)",
         "config": {"workload": wl.name, "desc": wl.desc, "tensors_per_rank": T,
                    "launch": "one CUDA graph per step" if args.graph else "direct launches",
                    "codebooks": "reused from a calibration plan (no histogram pass per step)" if args.reuse
@@ -445,19 +504,133 @@ def run_ours(args, rank, world, device):
                    else "contiguous tensors",
                    "raw_blocks": bool(args.raw_blocks),
                    "raw_bytes_per_rank": wl.raw_bytes, "mode": "one batch" if args.mode == "batch" else "per layer",
-                   "l2": "inputs larger than L2 (%.2f GB per step per rank)" % (wl.raw_bytes / 1e9),
+                   "l2": "inputs larger than L2, no flush (%.2f GB per step per rank)" % (wl.raw_bytes / 1e9),
                    "parallelism": "replicas" if world == 1 else "dp%d (independent tensors)" % world},
+        "step_stats": {"replays": reps, "median_ms": round(statistics.median(more), 4),
+                       "p10_ms": round(more[reps // 10], 4), "p90_ms": round(more[(9 * reps) // 10], 4),
+                       "value_at_median": round(wl.raw_bytes / (statistics.median(more) * 1e-3) / 1e9, 2),
+                       "timed_steps_median_ms": round(statistics.median(step_ms), 4)},
         "encode_gbs": round(wl.raw_bytes / ((t_plan + t_enc) * 1e-3) / 1e9, 1),
         "decode_gbs": round(wl.raw_bytes / (t_dec * 1e-3) / 1e9, 1),
         "ratio": round(wl.raw_bytes / stream_bytes, 5),
         "escape_fraction": round(E_total / sum(wl.n), 6),
-        "kernels": {k: {"ms": round(v["ms"], 4), "gbs": round(v["gbs"], 1), "frac": round(v["frac"], 4)}
+        "kernels": {k: {kk: (round(vv, 4) if kk != "gbs" else round(vv, 1)) for kk, vv in v.items()}
                     for k, v in kern.items()},
         "roofline": roof,
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
     return res, wl
+
+
+# ------------------------------------------------------ per-config records
+
+L2_FLUSH_BYTES = 256 << 20   # written between measurements that must start with a cold L2 (2x its 126 MB)
+
+
+def record_of(res: dict) -> dict:
+    """The figures of one workload's run (run_ours) for the `configs` object."""
+    keep = ("value", "unit", "ms_per_step", "ratio", "escape_fraction", "encode_gbs", "decode_gbs",
+            "kernels", "roofline", "step_stats", "gpu_launches", "clocks")
+    out = {"workload": res["config"]["workload"], "desc": res["config"]["desc"],
+           "mode": res["config"]["mode"], "l2": res["config"]["l2"], "dtype": res["dtype"]}
+    out.update({k: res[k] for k in keep if k in res})
+    return out
+
+
+def record_qwen3_stream(args, device, peak: float, peak_kind: str, layers: int = None) -> dict:
+    """Qwen3-32B KV at 131072 tokens, as the config describes it: 64 layers x
+    {K, V} x [131072, 8, 128] bf16 (34.4 GB), generated on the device one layer
+    at a time and coded layer by layer -- plan, encode and decode of the layer's
+    K and V, one batched call each (537 MB per call).  Before each layer's
+    measured pass a 256 MB buffer is written, so that the layer starts with a
+    cold L2 (`cold`); the same calls are then repeated at once (`warm`: L2 holds
+    what the first pass left).  Per-kernel figures are medians over the layers;
+    every layer's decode is checked bit for bit against its input."""
+    import fp8_kv_cache_exp_b200 as sz
+    cfg = kvgen.CONFIGS["qwen3-32b"]
+    nl = cfg.layers if layers is None else layers
+    n = cfg.numel
+    stream = torch.cuda.current_stream()
+    ws = sz.new_workspace(0, [n, n])
+    plans = sz.new_plans(2)
+    outs = [torch.empty(sz.sz_max_compressed_size(0, n), dtype=torch.uint8, device=device) for _ in range(2)]
+    decs = [torch.empty(cfg.shape, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    raw_layer = 2 * n * 2
+    names = ("plan", "encode", "decode")
+    cold = {k: [] for k in names}
+    warm = {k: [] for k in names}
+    kb = {k: [] for k in names}
+    stream_total = E_total = 0
+    clocks = ClockSampler(gpu_uuid(device))
+    clocks.start()
+    for layer in range(nl):
+        xs = [kvgen.kv_tensor(cfg, layer, kv, device=device) for kv in (0, 1)]
+        b = sz.Batch(0, xs, outs, ws, plans, decs=decs)
+        if layer == 0:  # first calls of these sizes (launch setup), not measured
+            b.plan(); b.encode(); b.decode()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+        head_start()
+        flush.fill_(layer & 0xFF)
+        for rep in range(2):
+            ev[4 * rep].record(stream)
+            b.plan()
+            ev[4 * rep + 1].record(stream)
+            b.encode()
+            ev[4 * rep + 2].record(stream)
+            b.decode()
+            ev[4 * rep + 3].record(stream)
+        torch.cuda.synchronize()
+        check_status(sz, [ws], "qwen3-32b layer %d" % layer)
+        for x, d in zip(xs, decs):
+            if not torch.equal(x.view(torch.uint8), d.view(torch.uint8)):
+                raise RuntimeError("qwen3-32b layer %d: round trip mismatch" % layer)
+        heads = torch.stack([o[:64] for o in outs]).cpu()
+        sb = int(heads[:, 40:48].contiguous().view(torch.int64).sum().item())
+        E_total += int(heads[:, 16:24].contiguous().view(torch.int64).sum().item())
+        stream_total += sb
+        layer_bytes = {"plan": raw_layer + 128, "encode": raw_layer + sb, "decode": raw_layer + sb}
+        for i, k in enumerate(names):
+            cold[k].append(ev[i].elapsed_time(ev[i + 1]))
+            warm[k].append(ev[4 + i].elapsed_time(ev[4 + i + 1]))
+            kb[k].append(layer_bytes[k])
+        del xs, b
+    clk = clocks.stop()
+    del flush, outs, decs, ws
+    torch.cuda.empty_cache()
+
+    kern = {}
+    for k in names:
+        g_cold = [by / (t * 1e-3) / 1e9 for by, t in zip(kb[k], cold[k])]
+        g_warm = [by / (t * 1e-3) / 1e9 for by, t in zip(kb[k], warm[k])]
+        kern[k] = {"ms": round(statistics.median(cold[k]), 4), "gbs": round(statistics.median(g_cold), 1),
+                   "frac": round(statistics.median(g_cold) / peak, 4),
+                   "frac_min": round(min(g_cold) / peak, 4), "frac_max": round(max(g_cold) / peak, 4),
+                   "warm_ms": round(statistics.median(warm[k]), 4),
+                   "warm_frac": round(statistics.median(g_warm) / peak, 4)}
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    t_cold = sum(sum(cold[k]) for k in names)
+    raw_all = raw_layer * nl
+    return {
+        "workload": "qwen3-32b", "desc": "Qwen3-32B KV at 131072 tokens: %d layers x {K,V} x [131072,8,128] bf16, "
+                                         "generated on the device and coded layer by layer (537 MB per call)" % nl,
+        "mode": "per layer, streamed", "dtype": "u16", "layers": nl,
+        "l2": "cold: 256 MB written before each layer (inputs 537 MB per layer); warm: the layer's calls repeated",
+        "value": round(raw_all / (t_cold * 1e-3) / 1e9, 2), "unit": UNIT,
+        "ms_per_layer": round(t_cold / nl, 4),
+        "ratio": round(raw_all / stream_total, 5), "escape_fraction": round(E_total / (2 * n * nl), 6),
+        "encode_gbs": round(raw_layer / ((kern["plan"]["ms"] + kern["encode"]["ms"]) * 1e-3) / 1e9, 1),
+        "decode_gbs": round(raw_layer / (kern["decode"]["ms"] * 1e-3) / 1e9, 1),
+        "kernels": kern,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": kern[dom]["frac"], "traffic": profiled_traffic(dom + "_kernel", "qwen3-32b"),
+                     "algorithmic_bytes": int(statistics.median(kb[dom])), "peak_source": peak_kind,
+                     "timing": "median over %d layers of one launch each, cold L2" % nl},
+        "gpu_launches": 3 * 2 * nl,
+        "clocks": clk,
+    }
 
 
 def run_transfer(args, wl, device, res):
@@ -634,47 +807,81 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def oracle_sample(cfg_name: str, budget_s: float, raw_blocks: bool = False):
-    """Time the CPU oracle (as it stands) on one layer's K and V (the stress
-    workload: a 2^23-element tensor of the same generator): plan + encode + decode."""
+class pinned_to_one_core:
+    """Pin this process to one host core (the highest-numbered one it may use)
+    for the duration of a with-block, then restore its affinity."""
+
+    def __enter__(self):
+        self.saved = None
+        self.core = None
+        try:
+            self.saved = os.sched_getaffinity(0)
+            self.core = max(self.saved)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            self.saved = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+
+def oracle_host_sample(cfg_name: str):
+    """(dtype, host byte arrays, description) of the reference arm's per-step
+    sample: one layer's K and V (the stress workload: a 2^23-element tensor of
+    the same generator)."""
+    if cfg_name == "stress-uniform":
+        xs = [kvgen.stress_tensor(STRESS_SAMPLE_N, None, stress_seed())]
+        return 0, [x.contiguous().view(torch.uint8).reshape(-1).numpy() for x in xs], \
+            "stress-uniform 2^23 elements"
+    cfg = kvgen.CONFIGS[cfg_name]
+    xs = [kvgen.kv_tensor(cfg, 0, kv) for kv in (0, 1)]
+    return (1 if cfg.fp8 else 0), [x.contiguous().view(torch.uint8).reshape(-1).numpy() for x in xs], \
+        "%s layer 0 K+V" % cfg_name
+
+
+def oracle_sample(dt: int, raws, what: str, budget_s: float, raw_blocks: bool = False, max_reps: int = 1 << 30):
+    """Time the CPU oracle (as it stands: plain single-threaded C), pinned to one
+    host core, on the tensors `raws` (host byte arrays): plan + encode + decode
+    of each, in order, repeated until budget_s seconds have passed (at least one
+    tensor, at most max_reps passes).  A pass that runs out of budget stops
+    after the tensor in progress; the sample says how many tensors were coded."""
     import numpy as np
     import oracle
-    if cfg_name == "stress-uniform":
-        dt = 0
-        xs = [kvgen.stress_tensor(STRESS_SAMPLE_N, None, stress_seed())]
-        what = "stress-uniform 2^23 elements"
-    else:
-        cfg = kvgen.CONFIGS[cfg_name]
-        dt = 1 if cfg.fp8 else 0
-        xs = [kvgen.kv_tensor(cfg, 0, kv) for kv in (0, 1)]
-        what = "%s layer 0 K+V" % cfg_name
-    raws = [x.contiguous().view(torch.uint8).reshape(-1).numpy() for x in xs]
-    nbytes = sum(r.size for r in raws)
     t_enc = t_dec = 0.0
+    coded = 0
+    nbytes = 0
     reps = 0
-    t_start = time.perf_counter()
-    while True:
-        for r in raws:
-            n = r.size // (2 if dt == 0 else 1)
-            t0 = time.perf_counter()
-            s = oracle.encode(dt, r, raw_blocks=raw_blocks)
-            t1 = time.perf_counter()
-            back = oracle.decode(s, n, dt)
-            t2 = time.perf_counter()
-            t_enc += t1 - t0
-            t_dec += t2 - t1
-            if not np.array_equal(back, r):
-                raise RuntimeError("oracle round trip mismatch")
-        reps += 1
-        if time.perf_counter() - t_start > budget_s:
-            break
-    raw_total = nbytes * reps
+    with pinned_to_one_core() as pin:
+        t_start = time.perf_counter()
+        done = False
+        while not done and reps < max_reps:
+            for r in raws:
+                n = r.size // (2 if dt == 0 else 1)
+                t0 = time.perf_counter()
+                s = oracle.encode(dt, r, raw_blocks=raw_blocks)
+                t1 = time.perf_counter()
+                back = oracle.decode(s, n, dt)
+                t2 = time.perf_counter()
+                t_enc += t1 - t0
+                t_dec += t2 - t1
+                if not np.array_equal(back, r):
+                    raise RuntimeError("oracle round trip mismatch")
+                coded += 1
+                nbytes += r.size
+                if time.perf_counter() - t_start > budget_s:
+                    done = True
+                    break
+            reps += 1
+        core = pin.core
     return {
-        "value": round(raw_total / (t_enc + t_dec) / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-        "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
-        "sample": "%s (%.1f MB raw) x %d rep(s), single-threaded C oracle%s" % (
-            what, nbytes / 1e6, reps, ", raw blocks allowed" if raw_blocks else ""),
-        "encode_gbs": round(raw_total / t_enc / 1e9, 4), "decode_gbs": round(raw_total / t_dec / 1e9, 4),
+        "value": round(nbytes / (t_enc + t_dec) / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "pinned_core": core, "host_cores": os.cpu_count(), "cpu_model": cpu_model(),
+        "sample": "%s: %d tensor(s) coded, %.1f MB raw, single-threaded C oracle pinned to one core%s" % (
+            what, coded, nbytes / 1e6, ", raw blocks allowed" if raw_blocks else ""),
+        "encode_gbs": round(nbytes / t_enc / 1e9, 4), "decode_gbs": round(nbytes / t_dec / 1e9, 4),
         "seconds": round(t_enc + t_dec, 2),
     }
 
@@ -683,19 +890,22 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     cfg_name = WORKLOADS[args.workload][0]
+    dt, raws, what = oracle_host_sample(cfg_name)
     sample = None
     times = []
     for k in range(args.warmup + args.steps):
-        r = oracle_sample(cfg_name, 0.0, args.raw_blocks)
+        r = oracle_sample(dt, raws, what, 0.0, args.raw_blocks, max_reps=1)
         if k >= args.warmup:
             times.append(r)
         sample = r
     val = statistics.median(t["value"] for t in times)
-    fp8 = cfg_name != "stress-uniform" and kvgen.CONFIGS[cfg_name].fp8
-    raw = STRESS_SAMPLE_N * 2 if cfg_name == "stress-uniform" else 2 * kvgen.CONFIGS[cfg_name].numel * (1 if fp8 else 2)
+    fp8 = dt == 1
+    raw = sum(r.size for r in raws)
     ms = raw / (val * 1e9) * 1e3
     cpu = dict(sample)
     cpu["value"] = val
+    cpu["sample"] = "%s per step (%d steps, median), single-threaded C oracle pinned to one core" % (
+        what, args.steps)
     return {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
@@ -727,12 +937,18 @@ def main():
     ap.add_argument("--transfer", action="store_true",
                     help="also run the layer-pipelined transfer (encode on the source, decode on the destination)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
-                    help="time the step with direct launches instead of one captured CUDA graph per step "
-                         "(per-kernel times always come from direct launches)")
+                    help="time the step with direct launches instead of one captured CUDA graph per step")
     ap.add_argument("--raw-blocks", action="store_true",
                     help="allow raw blocks (header flag): blocks that would expand are stored raw")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--no-records", action="store_true",
+                    help="skip the other workloads' records (`configs`) of the default run")
+    ap.add_argument("--qwen3-layers", type=int, default=None,
+                    help="layers of the streamed Qwen3-32B record (default: all 64)")
+    ap.add_argument("--kernel-reps", type=int, default=50,
+                    help="replays of each kernel's graph for the per-kernel figures (at least --steps)")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=30.0,
+                    help="bound on the CPU oracle's timed work (0: skip it)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -762,9 +978,35 @@ def main():
             res["e2e"] = e2e
         if args.transfer:
             res["transfer"] = run_transfer(args, wl, device, res)
-        if rank == 0 and world == 1 and args.cpu_baseline_seconds > 0:
-            res["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload][0], args.cpu_baseline_seconds,
-                                                args.raw_blocks)
+        default_run = (args.workload == "llama3-8b" and args.mode == "batch" and not args.reuse and
+                       not args.paged and not args.raw_blocks and args.layers is None and not args.transfer)
+        if world == 1 and default_run and not args.no_records:
+            # the other KV configurations, measured in the same run
+            peak, peak_kind = load_peaks()
+            recs = {}
+            a2 = argparse.Namespace(**vars(args))
+            a2.mode = "per_layer"
+            r, _ = run_ours(a2, rank, world, device, wl=wl)
+            recs["llama3-8b-per-layer"] = record_of(r)
+            hosts = [x.cpu() for x in wl.xs] if args.cpu_baseline_seconds > 0 else None
+            del wl
+            torch.cuda.empty_cache()
+            recs["qwen3-32b"] = record_qwen3_stream(args, device, peak, peak_kind, args.qwen3_layers)
+            a3 = argparse.Namespace(**vars(args))
+            a3.workload = "qwen3-30b-a3b-e5m2"
+            r, wl5 = run_ours(a3, rank, world, device)
+            recs["qwen3-30b-a3b-e5m2"] = record_of(r)
+            del wl5
+            torch.cuda.empty_cache()
+            res["configs"] = recs
+            if hosts is not None:
+                raws = [h.contiguous().view(torch.uint8).reshape(-1).numpy() for h in hosts]
+                res["cpu_baseline"] = oracle_sample(0, raws, "llama3-8b, all 64 K/V tensors of the batch",
+                                                    args.cpu_baseline_seconds, max_reps=1)
+        elif rank == 0 and world == 1 and args.cpu_baseline_seconds > 0:
+            dt, raws, what = oracle_host_sample(WORKLOADS[args.workload][0])
+            res["cpu_baseline"] = oracle_sample(dt, raws, what, args.cpu_baseline_seconds, args.raw_blocks,
+                                                max_reps=30)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

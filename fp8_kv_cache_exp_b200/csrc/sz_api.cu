@@ -140,13 +140,13 @@ sz_status sz_plan_set_flags(int T, sz_plan_t *d_plans, unsigned flags, cudaStrea
     return SZ_OK;
 }
 
-namespace {
+}  // extern "C"
 
-// Ordinary encode (plans are the tensors' own) or codebook reuse (plans give
-// codebooks only).
-sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
-                        const uint64_t *n, void *const *d_out, const size_t *out_cap, uint64_t *d_totals,
-                        bool reuse, const sz_paged_t *paged, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+namespace sz {
+
+sz_status check_encode_args(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
+                            const uint64_t *n, void *const *d_out, const size_t *out_cap, const uint64_t *d_totals,
+                            const void *d_ws, size_t ws_bytes) {
     sz_status s = check_batch(dtype, T, n, d_ws, ws_bytes);
     if (s != SZ_OK) return s;
     if (!d_plans || !aligned(d_plans, 8) || !d_in || !d_out || !out_cap) return SZ_ERR_INVALID_ARG;
@@ -157,6 +157,22 @@ sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const v
         // the smallest stream for n (no escapes) must fit in any case
         if (out_cap[t] < stream_layout(dtype, n[t], 0).total) return SZ_ERR_BUFFER_TOO_SMALL;
     }
+    return SZ_OK;
+}
+
+}  // namespace sz
+
+extern "C" {
+
+namespace {
+
+// Ordinary encode (plans are the tensors' own) or codebook reuse (plans give
+// codebooks only).
+sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
+                        const uint64_t *n, void *const *d_out, const size_t *out_cap, uint64_t *d_totals,
+                        bool reuse, const sz_paged_t *paged, void *d_ws, size_t ws_bytes, cudaStream_t stream) {
+    const sz_status s = check_encode_args(dtype, T, d_plans, d_in, n, d_out, out_cap, d_totals, d_ws, ws_bytes);
+    if (s != SZ_OK) return s;
     const uint64_t tiles = total_tiles(T, n);
     const WsLayout w = ws_layout(T, tiles);
     uint8_t *ws = static_cast<uint8_t *>(d_ws);

@@ -132,8 +132,8 @@ __host__ __device__ inline Layout stream_layout(int dtype, uint64_t n, uint64_t 
 struct WsLayout {
     size_t hist, ticket, status, bytes;
 };
-inline WsLayout ws_layout(int T, uint64_t total_tiles) {
-    WsLayout w;
+constexpr WsLayout ws_layout(int T, uint64_t total_tiles) {
+    WsLayout w{};
     w.hist = kCtlWords * 4;
     w.ticket = w.hist + size_t(T) * 256 * 4;
     w.status = w.ticket + align256(size_t(T) * 4);

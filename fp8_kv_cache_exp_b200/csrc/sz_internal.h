@@ -42,6 +42,13 @@ struct DecodeArgs {
     const sz_paged_t *paged;  // T output page descriptors, or null (contiguous outputs)
 };
 
+// Host checks of an encode call (contiguous or paged inputs; the pools of
+// paged ones in d_in) against the workspace at d_ws: SZ_OK, or the status the
+// call returns without enqueuing anything.
+sz_status check_encode_args(sz_dtype dtype, int T, const sz_plan_t *d_plans, const void *const *d_in,
+                            const uint64_t *n, void *const *d_out, const size_t *out_cap, const uint64_t *d_totals,
+                            const void *d_ws, size_t ws_bytes);
+
 // Kernel page reference of descriptor d (or a contiguous tensor when d is null).
 PageRef page_ref(const sz_paged_t *d);
 

@@ -15,14 +15,16 @@
 
 #include "splitzip.h"
 #include "sz_common.cuh"
+#include "sz_internal.h"
 
 namespace {
 
 // Largest tensor this entry point accepts, and the scratch it needs: the
-// workspace of one tensor (control block, histogram, ticket, one look-back
-// status word per 4096-element tile).
+// workspace of one tensor of that size (control block, histogram, ticket, one
+// look-back status word per 4096-element tile) -- 263,680 bytes.
 constexpr uint64_t kNoAllocMaxTiles = SZ_NOALLOC_MAX_ELEMS / sz::kBlock;
-constexpr size_t kNoAllocScratchBytes = 256 + 1024 + 256 + 8 * kNoAllocMaxTiles;
+constexpr size_t kNoAllocScratchBytes = sz::ws_layout(1, kNoAllocMaxTiles).bytes;
+static_assert(kNoAllocScratchBytes == 263680, "the header states the scratch size");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -33,9 +35,7 @@ std::atomic<void *> g_scratch_ptr[kMaxDevices];
 // Device address of the scratch array on the current device.  The host-side
 // name g_noalloc_scratch is only a stand-in; the address is looked up once per
 // device, with that device current, and cached.
-sz_status scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SZ_ERR_CUDA;
+sz_status scratch_address(int dev, void **out) {
     void *p = g_scratch_ptr[dev].load(std::memory_order_acquire);
     if (p == nullptr) {
         std::lock_guard<std::mutex> lock(g_setup_mutex);
@@ -57,14 +57,30 @@ extern "C" sz_status sz_encode_noalloc(sz_dtype dtype, const sz_plan_t *d_plan, 
                                        uint32_t *d_status, cudaStream_t stream) {
     if (dtype != SZ_BF16 && dtype != SZ_FP8_E5M2) return SZ_ERR_UNSUPPORTED_DTYPE;
     if (n > SZ_NOALLOC_MAX_ELEMS) return SZ_ERR_BUFFER_TOO_SMALL;  // beyond the static scratch
+    if (d_status != nullptr && (reinterpret_cast<uintptr_t>(d_status) & 3u) != 0) return SZ_ERR_INVALID_ARG;
+    // The scratch used is the current device's: a stream of another device
+    // would run the kernel there against this device's array, so it is refused.
+    int dev = 0, stream_dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SZ_ERR_CUDA;
+    // (the default streams always belong to the current device)
+    if (stream != nullptr && stream != cudaStreamLegacy && stream != cudaStreamPerThread) {
+        if (cudaStreamGetDevice(stream, &stream_dev) != cudaSuccess) return SZ_ERR_INVALID_ARG;
+        if (stream_dev != dev) return SZ_ERR_INVALID_ARG;
+    }
     void *scratch = nullptr;
-    sz_status s = scratch_address(&scratch);
+    sz_status s = scratch_address(dev, &scratch);
+    if (s != SZ_OK) return s;
+    const size_t ws_bytes = sz_workspace_bytes(dtype, n);
+    if (ws_bytes == 0 || ws_bytes > kNoAllocScratchBytes) return SZ_ERR_BUFFER_TOO_SMALL;
+    // Every argument check of sz_encode first, so that a call refused on the
+    // host enqueues nothing (not even the memset below).
+    const void *in[1] = {d_in};
+    void *out[1] = {d_out};
+    s = sz::check_encode_args(dtype, 1, d_plan, in, &n, out, &out_cap, nullptr, scratch, ws_bytes);
     if (s != SZ_OK) return s;
     // The scratch keeps the previous call's contents.  Zero the control block
     // (error word, job and done counters) and this call's look-back status
     // words, which the kernel expects to start at zero.
-    const size_t ws_bytes = sz_workspace_bytes(dtype, n);
-    if (ws_bytes == 0 || ws_bytes > kNoAllocScratchBytes) return SZ_ERR_BUFFER_TOO_SMALL;
     if (cudaMemsetAsync(scratch, 0, ws_bytes, stream) != cudaSuccess) return SZ_ERR_CUDA;
     s = sz_encode(dtype, d_plan, d_in, n, d_out, out_cap, scratch, ws_bytes, stream);
     if (s != SZ_OK) return s;

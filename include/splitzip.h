@@ -298,16 +298,19 @@ sz_status sz_last_device_status(void *d_ws, cudaStream_t stream);
  * example an engine that reserves all of the GPU's memory for its KV pool at
  * start-up and hands the codec only the tensor, the destination buffer and a
  * stream.  The call runs the same kernel as sz_encode on a scratch area held
- * by the library: a static device array of 262,400 bytes (enough for
- * SZ_NOALLOC_MAX_ELEMS elements) that every GPU which loads the library keeps
- * until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * by the library: a static device array of 263,680 bytes (the workspace of
+ * one tensor of SZ_NOALLOC_MAX_ELEMS elements) that every GPU which loads the
+ * library keeps until the process exits.  It calls no cudaMalloc, cudaFree or other
  * allocating routine; it enqueues a memset of the scratch it uses, the encode
  * kernel and, if d_status is not NULL, a 4-byte device-to-device copy.
  *
- * Arguments are those of sz_encode; d_status (device, may be NULL) receives
- * the call's device error word (SZ_OK or a device-found error) once the
- * stream reaches it.  n > SZ_NOALLOC_MAX_ELEMS returns SZ_ERR_BUFFER_TOO_SMALL
- * at once, with nothing enqueued.
+ * Arguments are those of sz_encode; d_status (device, 4-byte aligned, may be
+ * NULL) receives the call's device error word (SZ_OK or a device-found error)
+ * once the stream reaches it.  n > SZ_NOALLOC_MAX_ELEMS returns
+ * SZ_ERR_BUFFER_TOO_SMALL, and every other host check of sz_encode its
+ * status, at once and with nothing enqueued.  The scratch used is the current
+ * device's: a stream that belongs to another device is refused
+ * (SZ_ERR_INVALID_ARG).
  *
  * The first call on each device looks up the scratch array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call

@@ -29,3 +29,23 @@ def test_reference_arm_line_on_cpu():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     import bench
     assert line["metric"] == bench.METRIC
+
+
+def test_oracle_pinning_restores_affinity():
+    """The CPU baseline runs pinned to one host core and leaves the process's
+    affinity as it found it."""
+    import os
+    import bench
+    before = os.sched_getaffinity(0)
+    with bench.pinned_to_one_core() as pin:
+        assert os.sched_getaffinity(0) == {pin.core}
+        assert pin.core in before
+    assert os.sched_getaffinity(0) == before
+
+
+def test_kernel_figures_mean_and_median():
+    import bench
+    f = bench.kernel_figures([1.0, 2.0, 6.0], 3e9, 1000.0)
+    assert abs(f["ms"] - 3.0) < 1e-12 and f["ms_median"] == 2.0
+    assert abs(f["gbs"] - 1000.0) < 1e-9 and abs(f["frac"] - 1.0) < 1e-12
+    assert abs(f["frac_median"] - 1.5) < 1e-12
