@@ -528,6 +528,14 @@ def run_ours(args, rank, world, device, wl=None):
 L2_FLUSH_BYTES = 256 << 20   # written between measurements that must start with a cold L2 (2x its 126 MB)
 
 
+def cold_l2(buf: torch.Tensor, tag: int = 0):
+    """Leave L2 holding none of the data that follows and no dirty lines: write
+    a buffer of twice its size (evicting everything, writing back what was
+    dirty), then read it (the written lines go back to DRAM, clean copies stay)."""
+    buf.fill_(tag & 0xFF)
+    buf.view(torch.int32).sum()
+
+
 def record_of(res: dict) -> dict:
     """The figures of one workload's run (run_ours) for the `configs` object."""
     keep = ("value", "unit", "ms_per_step", "ratio", "escape_fraction", "encode_gbs", "decode_gbs",
@@ -543,8 +551,8 @@ def record_qwen3_stream(args, device, peak: float, peak_kind: str, layers: int =
     {K, V} x [131072, 8, 128] bf16 (34.4 GB), generated on the device one layer
     at a time and coded layer by layer -- plan, encode and decode of the layer's
     K and V, one batched call each (537 MB per call).  Before each layer's
-    measured pass a 256 MB buffer is written, so that the layer starts with a
-    cold L2 (`cold`); the same calls are then repeated at once (`warm`: L2 holds
+    measured pass a 256 MB buffer is written and read back, so that the layer
+    starts with a cold L2 holding no dirty lines (`cold`); the same calls are then repeated at once (`warm`: L2 holds
     what the first pass left).  Per-kernel figures are medians over the layers;
     every layer's decode is checked bit for bit against its input."""
     import fp8_kv_cache_exp_b200 as sz
@@ -573,7 +581,7 @@ def record_qwen3_stream(args, device, peak: float, peak_kind: str, layers: int =
         torch.cuda.synchronize()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
         head_start()
-        flush.fill_(layer & 0xFF)
+        cold_l2(flush, layer)
         for rep in range(2):
             ev[4 * rep].record(stream)
             b.plan()
@@ -617,7 +625,8 @@ def record_qwen3_stream(args, device, peak: float, peak_kind: str, layers: int =
         "workload": "qwen3-32b", "desc": "Qwen3-32B KV at 131072 tokens: %d layers x {K,V} x [131072,8,128] bf16, "
                                          "generated on the device and coded layer by layer (537 MB per call)" % nl,
         "mode": "per layer, streamed", "dtype": "u16", "layers": nl,
-        "l2": "cold: 256 MB written before each layer (inputs 537 MB per layer); warm: the layer's calls repeated",
+        "l2": "cold: 256 MB written and read back before each layer (inputs 537 MB per layer); "
+                    "warm: the layer's calls repeated at once",
         "value": round(raw_all / (t_cold * 1e-3) / 1e9, 2), "unit": UNIT,
         "ms_per_layer": round(t_cold / nl, 4),
         "ratio": round(raw_all / stream_total, 5), "escape_fraction": round(E_total / (2 * n * nl), 6),

@@ -40,16 +40,29 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, extra_flags=(), out: str = LIB, verbose: bool = False) -> str:
-    """Compile every csrc/*.cu into one shared library; return its path."""
+    """Compile every csrc/*.cu (one nvcc per file, in parallel) and link them
+    into one shared library; return its path."""
     if not force and out == LIB and up_to_date():
         return out
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = out + ".tmp.%d" % os.getpid()
-    cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp,
-           *sources()]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
+    with tempfile.TemporaryDirectory(prefix="splitzip_build_") as objdir:
+        def compile_one(src):
+            obj = os.path.join(objdir, os.path.basename(src) + ".o")
+            cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+            if verbose:
+                print(" ".join(cmd))
+            subprocess.run(cmd, check=True)
+            return obj
+        srcs = sources()
+        with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+            objs = list(ex.map(compile_one, srcs))
+        cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
+        if verbose:
+            print(" ".join(cmd))
+        subprocess.run(cmd, check=True)
     os.replace(tmp, out)
     return out
 
