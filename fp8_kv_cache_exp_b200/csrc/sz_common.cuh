@@ -13,6 +13,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "splitzip.h"
 
@@ -214,11 +215,46 @@ struct DecodeParams {
 // costs a claim, a look-back and a ring restart, so chunks stay as long as the
 // launch allows: a large batch keeps 8-block chunks, one layer's K and V
 // (4096 BF16 or 8192 E5M2 blocks) gets 2- or 4-block chunks and still spreads
-// over every SM (measured best for both).
+// over every SM (measured best for both; 1-block chunks for one Llama-3-8B
+// layer took 25% longer).
 inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_warps) {
     int lg = kMaxChunkLog2;
     while (lg > 0 && (total_blocks >> lg) < resident_warps / 2) --lg;
     return lg;
+}
+
+// ------------------------------------------------ programmatic dependent launch
+// The plan and decode kernels are launched with programmatic stream
+// serialization: each may start while the kernel before it on the stream is
+// still running (after that kernel's CTAs have all called
+// pdl_launch_dependents, or exited).  Before griddepcontrol.wait returns, a
+// kernel touches nothing but its parameters and its shared memory; the wait
+// returns once every kernel before it on the stream has completed and its
+// memory is visible.  So a launch's fixed costs (launch, CTA placement,
+// shared-memory set-up) overlap the previous kernel's tail, and the order of
+// memory effects is that of plain stream order.  The encode kernel waits in
+// the same way, so it is safe under either kind of launch; it is launched the
+// ordinary way (see its launcher).
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// Launch kern<<<grid, block, smem, stream>>>(args...) with programmatic stream
+// serialization allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                              cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------- device helpers

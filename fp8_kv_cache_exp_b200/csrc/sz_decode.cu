@@ -37,8 +37,13 @@ namespace sz {
 
 namespace {
 
-constexpr int NT = kTileThreads;
+// One CTA per SM of 24 independent warps (80 registers): every SM gets the
+// same number of warps however the CTAs are placed (see the encode kernel).
+constexpr int NT = 768;
 constexpr int NW = NT / 32;
+// The raw-block pass: one ordinary CTA per tensor.
+constexpr int kRawThreads = kTileThreads;
+constexpr int kRawWarps = kRawThreads / 32;
 constexpr int kStages = 4;                            // ring of input-unit stages per warp
 constexpr uint64_t kWaitLimitNs = 1000000000ull;      // 1 s
 
@@ -600,6 +605,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
         fence_mbar_init();
     }
     __syncwarp();
+    pdl_wait();  // nothing above touches global memory (programmatic launch)
+    pdl_launch_dependents();
 
     // Blocks are claimed one at a time from per-tensor counters, one block
     // ahead of the one being decoded.  Each warp starts in the tensor that
@@ -764,15 +771,15 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
     }
 }
 
-// Contiguous outputs: ptxas keeps this kernel at 80 registers on its own.
+// Contiguous outputs (80 registers: 24 warps per SM).
 template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT) decode_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
+__global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
     decode_body<DT, MAXB, false>(p);
 }
 
-// Paged outputs: capped for three CTAs per SM.
+// Paged outputs: capped at 80 registers like the contiguous kernel.
 template <int DT, int MAXB>
-__global__ void __launch_bounds__(NT, 3) decode_kernel_paged(const __grid_constant__ DecodeParams<MAXB> p) {
+__global__ void __launch_bounds__(NT, 1) decode_kernel_paged(const __grid_constant__ DecodeParams<MAXB> p) {
     decode_body<DT, MAXB, true>(p);
 }
 
@@ -782,17 +789,19 @@ __global__ void __launch_bounds__(NT, 3) decode_kernel_paged(const __grid_consta
 // stream without the flag costs one header read.  Keeping raw blocks out of
 // those kernels' loops keeps the loops as fast as without them (measured).
 template <int DT, int MAXB, bool PAGED>
-__global__ void __launch_bounds__(NT) raw_pass_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
-    __shared__ uint32_t s_tab[NW][256];
+__global__ void __launch_bounds__(kRawThreads) raw_pass_kernel(const __grid_constant__ DecodeParams<MAXB> p) {
+    __shared__ uint32_t s_tab[kRawWarps][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = int(blockIdx.x);
+    pdl_wait();
+    pdl_launch_dependents();
     if (t >= p.T || p.n[t] == 0) return;
     WarpStream ws;
     warp_open_stream<DT, MAXB>(p, t, s_tab[warp], ws);  // each warp, for its own copy of ws
     if (!ws.ok || !ws.raw_ok) return;
     const uint8_t *comp = p.comp[t];
     const uint32_t *tabw = reinterpret_cast<const uint32_t *>(comp + 64);
-    for (uint32_t b0 = uint32_t(warp) * 32; b0 < ws.nb; b0 += NW * 32) {
+    for (uint32_t b0 = uint32_t(warp) * 32; b0 < ws.nb; b0 += kRawWarps * 32) {
         const uint32_t b = b0 + uint32_t(lane);
         bool raw = false;
         uint32_t lo = 0;
@@ -835,13 +844,15 @@ sz_status launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     }
     p.total_blocks = p.block_begin[a.T];
     if (p.total_blocks == 0) return SZ_OK;
-    // enough CTAs to fill the GPU, but no more warps than blocks
+    // a CTA per SM (fewer only if there are fewer blocks than SMs); warps claim blocks
     const uint64_t resident = uint64_t(a.num_sms) * per_sm;
-    const uint64_t need = cdiv(p.total_blocks, NW);
-    const uint64_t grid = need < resident ? need : resident;
-    kern<<<unsigned(grid), NT, smem, stream>>>(p);
-    if (PAGED || DT == SZ_FP8_E5M2) raw_pass_kernel<DT, MAXB, PAGED><<<unsigned(a.T), NT, 0, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+    const uint64_t grid = p.total_blocks < resident ? p.total_blocks : resident;
+    if (launch_pdl(kern, unsigned(grid), NT, smem, stream, p) != cudaSuccess) return SZ_ERR_CUDA;
+    if (PAGED || DT == SZ_FP8_E5M2)
+        return launch_pdl(raw_pass_kernel<DT, MAXB, PAGED>, unsigned(a.T), kRawThreads, 0, stream, p) == cudaSuccess
+                   ? SZ_OK
+                   : SZ_ERR_CUDA;
+    return SZ_OK;
 }
 
 }  // namespace

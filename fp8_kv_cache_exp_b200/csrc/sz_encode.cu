@@ -35,13 +35,17 @@ namespace sz {
 
 namespace {
 
+// Persistent CTAs of 8 independent warps: 3 per SM at 80 registers (BF16), 2
+// per SM at 128 registers (E5M2 does more work per loaded byte and runs faster
+// with more registers).  Measured against one CTA of 24 (16) warps per SM:
+// the same on large batches, slower on one Qwen3-32B layer (0.70 against
+// 0.76 of the HBM peak).
 constexpr int NT = kTileThreads;
 constexpr int NW = NT / 32;
 constexpr int kChunkBlocks = kMaxChunkBlocks;         // a warp's unit of work: up to 8 consecutive blocks
 constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per chunk (two chunks)
 constexpr int kRing = 3;                              // input-unit stages per warp
 constexpr uint32_t kUnitBytes = 2048;                 // one input unit: a quarter block (BF16) or half a block (E5M2)
-constexpr int kLookbackPerLane = 4;                   // status words per lane per step
 constexpr uint64_t kLookbackLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr uint64_t kWaitLimitNs = 1000000000ull;      // bulk-copy wait limit
 constexpr unsigned long long kFlagAgg = 1ull << 32;   // chunk aggregate published
@@ -70,10 +74,13 @@ struct Geo {
 // publishes the chunk's aggregate, then sums its predecessors' published
 // values back to the nearest inclusive prefix.  Status word: epoch (30 bits)
 // << 34 | flag << 32 | value; words of earlier launches carry an older epoch
-// and read as "not published".  Lane l reads positions 4l..4l+3 behind the
-// cursor (position 0 = nearest predecessor).  Every predecessor publishes its
-// aggregate as soon as it has coded its chunk, without waiting on anything, so
-// a look-back always ends; the total wait is still bounded (SZ_ERR_TIMEOUT).
+// and read as "not published".  A round reads the 128 nearest unsummed
+// predecessors (lane l: positions 4l .. 4l + 3 behind the cursor, position 0
+// = nearest).  Every predecessor publishes its aggregate as soon as it has
+// coded its chunk, without waiting on anything, so a look-back always ends;
+// the total wait is still bounded (SZ_ERR_TIMEOUT).  (Wider rounds were
+// measured: 512 predecessors per round made every encode slower, since a
+// deferred look-back is retried between the blocks of the warp's next chunk.)
 struct Lookback {
     int32_t j;      // nearest predecessor not yet summed
     uint32_t excl;  // escapes summed so far
@@ -81,6 +88,7 @@ struct Lookback {
     uint32_t flags; // kLbDone | kLbTimedOut | kLbWaiting
 };
 constexpr uint32_t kLbDone = 1, kLbTimedOut = 2, kLbWaiting = 4;
+constexpr int kLookbackPerLane = 4;  // status words per lane per round
 
 __device__ __forceinline__ void lookback_start(Lookback &lb, unsigned long long *st, uint32_t chunk,
                                                uint32_t agg, unsigned long long tag) {
@@ -98,33 +106,35 @@ __device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t 
     const int lane = threadIdx.x & 31;
     uint32_t backoff = 32;
     while (!(lb.flags & kLbDone)) {
-        uint32_t f[kLookbackPerLane], v[kLookbackPerLane];
+        constexpr int w = kLookbackPerLane;
+        unsigned long long word[w];
 #pragma unroll
-        for (int q = 0; q < kLookbackPerLane; ++q) {
-            const int32_t idx = lb.j - kLookbackPerLane * lane - q;
-            f[q] = 2;  // before chunk 0: a virtual inclusive prefix of 0
-            v[q] = 0;
-            if (idx >= 0) {
-                const unsigned long long w = ld_relaxed_u64(st + idx);
-                f[q] = ((w >> 34) == (tag >> 34)) ? uint32_t(w >> 32) & 3u : 0u;
-                v[q] = uint32_t(w);
+        for (int q = 0; q < w; ++q) {
+            const int32_t idx = lb.j - w * lane - q;
+            word[q] = idx >= 0 ? ld_relaxed_u64(st + idx) : 0ull;
+        }
+        // this lane's positions up to and including its nearest inclusive prefix
+        // (all w of them if it has none): their sum and whether all are published
+        int my_inc = w;
+        uint32_t sum = 0;
+        bool ready = true;
+#pragma unroll
+        for (int q = 0; q < w; ++q) {
+            if (my_inc == w) {
+                const int32_t idx = lb.j - w * lane - q;
+                // before chunk 0: a virtual inclusive prefix of 0
+                const uint32_t f = idx < 0 ? 2u
+                                           : (((word[q] >> 34) == (tag >> 34)) ? uint32_t(word[q] >> 32) & 3u : 0u);
+                sum += idx < 0 ? 0u : uint32_t(word[q]);
+                ready = ready && f != 0;
+                if (f == 2) my_inc = q;
             }
         }
-        int my_inc = kLookbackPerLane;  // this lane's nearest inclusive position
-#pragma unroll
-        for (int q = kLookbackPerLane - 1; q >= 0; --q)
-            if (f[q] == 2) my_inc = q;
-        const uint32_t inc_lanes = __ballot_sync(0xffffffffu, my_inc < kLookbackPerLane);
+        const uint32_t inc_lanes = __ballot_sync(0xffffffffu, my_inc < w);
         const int L = inc_lanes ? __ffs(inc_lanes) - 1 : 32;
-        const int need = lane < L ? kLookbackPerLane : (lane == L ? my_inc + 1 : 0);
-        bool ready = true;
-        uint32_t sum = 0;
-#pragma unroll
-        for (int q = 0; q < kLookbackPerLane; ++q) {
-            if (q < need) {
-                ready = ready && f[q] != 0;
-                sum += v[q];
-            }
+        if (lane > L) {  // past the nearest inclusive prefix: not needed
+            sum = 0;
+            ready = true;
         }
         if (__all_sync(0xffffffffu, ready)) {
             lb.excl += __reduce_add_sync(0xffffffffu, sum);
@@ -132,7 +142,7 @@ __device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t 
                 lb.flags |= kLbDone;
                 break;
             }
-            lb.j -= 32 * kLookbackPerLane;
+            lb.j -= 32 * w;
             continue;
         }
         const uint32_t now = __shfl_sync(0xffffffffu, uint32_t(global_ns()), 0);
@@ -817,24 +827,23 @@ __device__ __forceinline__ unsigned long long *chunk_status(const EncodeParams<M
     return p.status + p.chunk_begin[t];
 }
 
-// BF16: 3 CTAs per SM (80 registers).  E5M2 does more work per loaded byte and
-// runs faster with 2 CTAs per SM and 128 registers (measured).
 template <int DT, int MAXB, bool PAGED, int LG>
 __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     extern __shared__ __align__(128) uint8_t s_raw[];
     WarpShared *s_warp = reinterpret_cast<WarpShared *>(s_raw);
     __shared__ uint32_t s_epoch;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
-    __syncthreads();
-    const uint32_t epoch = s_epoch;
-    const unsigned long long tag = (unsigned long long)(epoch & 0x3FFFFFFFu) << 34;
     WarpShared &W = s_warp[warp];
     if (lane == 0) {
         for (int i = 0; i < kRing; ++i) mbar_init(&W.bar[i], 1);
         fence_mbar_init();
     }
-    __syncwarp();
+    pdl_wait();  // nothing above touches global memory (programmatic launch)
+    pdl_launch_dependents();
+    if (tid == 0) s_epoch = ld_relaxed_u32(&p.ctl[kCtlEpoch]);
+    __syncthreads();
+    const uint32_t epoch = s_epoch;
+    const unsigned long long tag = (unsigned long long)(epoch & 0x3FFFFFFFu) << 34;
     RingState R = {0u, 0u, 0u, 0u};
     int plan_tensor = -1;
     Pending pend;
@@ -939,6 +948,9 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
         kern = kern_any;
         if (resident_per_sm(reinterpret_cast<const void *>(kern_any), NT, smem, cache_any) < 1) return SZ_ERR_CUDA;
     }
+    // An ordinary launch: with a programmatic one, a small launch's CTAs pile
+    // onto the SMs that the previous kernel frees first (3 per SM), and one
+    // Llama-3-8B layer's encode took 45% longer (measured).
     kern<<<unsigned(grid), NT, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }

@@ -328,6 +328,15 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
     const int tid = threadIdx.x;
     const uint32_t col = smem_u32(s_cols + (tid % (NT / 2)));
     const uint32_t inc = 1u << (16 * (tid / (NT / 2)));
+    const uint64_t lo = p.total_items * blockIdx.x / gridDim.x;
+    const uint64_t hi = p.total_items * (blockIdx.x + 1) / gridDim.x;
+    // shared-memory set-up overlaps the previous kernel (programmatic launch)
+    if (lo < hi) {
+        for (int i = tid; i < C::kBins * (NT / 2) / 4; i += NT)
+            reinterpret_cast<uint4 *>(s_cols)[i] = make_uint4(0, 0, 0, 0);
+    }
+    pdl_wait();
+    pdl_launch_dependents();
 
     // Plans of empty tensors: codebook of the 15 smallest values, E = 0.
     if (blockIdx.x == 0) {
@@ -344,10 +353,7 @@ __global__ void __launch_bounds__(NT, 1) plan_kernel(const __grid_constant__ Pla
         }
     }
 
-    const uint64_t lo = p.total_items * blockIdx.x / gridDim.x;
-    const uint64_t hi = p.total_items * (blockIdx.x + 1) / gridDim.x;
     if (lo >= hi) return;
-    for (int i = tid; i < C::kBins * (NT / 2) / 4; i += NT) reinterpret_cast<uint4 *>(s_cols)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
 
     int t = find_tensor<uint64_t, MAXB>(p.item_begin, p.T, lo);
@@ -424,8 +430,7 @@ sz_status launch_plan_t(const PlanArgs &a, cudaStream_t stream) {
     uint64_t grid = uint64_t(a.num_sms) * per_sm;
     if (p.total_items < grid) grid = p.total_items;
     if (grid == 0) grid = 1;  // only empty tensors: block 0 writes their plans
-    kern<<<unsigned(grid), NT, smem, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+    return launch_pdl(kern, unsigned(grid), NT, smem, stream, p) == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }
 
 }  // namespace
