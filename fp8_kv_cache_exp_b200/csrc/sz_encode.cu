@@ -15,8 +15,8 @@
 //      lane has two) and staged in element order in the warp's stage;
 //   3. the chunk's escape offset comes from a single-pass decoupled look-back
 //      over the chunks of its tensor (128 predecessors per step, resumable; a
-//      chunk whose predecessors have not yet published is finished between the
-//      blocks of the warp's next chunk; every wait is bounded: SZ_ERR_TIMEOUT
+//      chunk whose predecessors have not yet published is finished once the
+//      warp has coded its next chunk; every wait is bounded: SZ_ERR_TIMEOUT
 //      instead of a hang);
 //   4. the chunk's offsets-table entries and escapes are written contiguously
 //      (a chunk whose escapes overflow the stage re-codes its input and writes
@@ -78,9 +78,11 @@ struct Geo {
 // predecessors (lane l: positions 4l .. 4l + 3 behind the cursor, position 0
 // = nearest).  Every predecessor publishes its aggregate as soon as it has
 // coded its chunk, without waiting on anything, so a look-back always ends;
-// the total wait is still bounded (SZ_ERR_TIMEOUT).  (Wider rounds were
-// measured: 512 predecessors per round made every encode slower, since a
-// deferred look-back is retried between the blocks of the warp's next chunk.)
+// the total wait is still bounded (SZ_ERR_TIMEOUT).  Measured variants: 512
+// predecessors per round made every encode slower; retrying a deferred
+// look-back between the blocks of the warp's next chunk (each try stalls the
+// warp for an L2 round trip) made the Llama-3-8B batch encode 4% and one
+// Qwen3-32B layer 8% slower than settling it once, after that chunk.
 struct Lookback {
     int32_t j;      // nearest predecessor not yet summed
     uint32_t excl;  // escapes summed so far
@@ -408,19 +410,12 @@ __device__ __forceinline__ uint32_t exponent_at(uint4 v, uint32_t j) {
     }
 }
 
-// Rank one step's escapes within the block and hand each to put(rank, exponent).
+// Escapes of a step in which some lane has two or more (rare on KV data):
+// a warp prefix of the per-lane counts c, then each lane hands its escapes
+// over in element order.  (Inline: as a call it made KV encode 23% slower,
+// measured.)
 template <int DT, typename Put>
-__device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &running, Put put) {
-    const uint32_t c = popc_mask(m);
-    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
-    if (any == 0) return;
-    if (__ballot_sync(0xffffffffu, c > 1) == 0) {
-        // at most one escape per lane: its rank counts the lanes before it that have one
-        const uint32_t lane = threadIdx.x & 31;
-        if (c) put(running + __popc(any & ((1u << lane) - 1u)), exponent_at<DT>(v, first_bit(m) >> 2));
-        running += __popc(any);
-        return;
-    }
+__device__ __forceinline__ void rank_general(EMask<DT> m, uint4 v, uint32_t c, uint32_t &running, Put put) {
     uint32_t tot;
     const uint32_t prefix = warp_exclusive_prefix(c, &tot);
     if (tot) {
@@ -432,6 +427,30 @@ __device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &runnin
         }
         running += tot;
     }
+}
+
+// Rank one step's escapes within the block and hand each to put(rank,
+// exponent).  With `wanted` false the escapes of a step with several per lane
+// are only counted: the caller has no room left for them (a chunk whose
+// escapes overflow its stage is coded again when it is finished, and its
+// escapes are written then).
+template <int DT, typename Put>
+__device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &running, Put put, bool wanted = true) {
+    const uint32_t c = popc_mask(m);
+    const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+    if (any == 0) return;
+    if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+        // at most one escape per lane: its rank counts the lanes before it that have one
+        const uint32_t lane = threadIdx.x & 31;
+        if (c) put(running + __popc(any & ((1u << lane) - 1u)), exponent_at<DT>(v, first_bit(m) >> 2));
+        running += __popc(any);
+        return;
+    }
+    if (!wanted) {
+        running += __reduce_add_sync(0xffffffffu, c);
+        return;
+    }
+    rank_general<DT>(m, v, c, running, put);
 }
 
 // One warp codes block blk of a tensor of n elements: planes and codes go to
@@ -484,48 +503,94 @@ __device__ __forceinline__ uint32_t code_block(uint32_t lut, const uint8_t *in, 
     return running;
 }
 
+// One lane's share of one step of a raw block (v: its up to LE elements, only
+// `valid` of them in the tensor): the low four bits of each exponent to the
+// code plane at cd (the bytes code_step wrote for this lane), the bits above
+// them to the escape section at h (BF16: a high nibble per element, E5M2: bit
+// 4 per element), bytes at or past bound not written.  A full step writes its
+// code bytes with one aligned store and its high bits with one store when h
+// is aligned for it.
+template <int DT>
+__device__ __forceinline__ void raw_step(uint4 v, int valid, uint8_t *cd, uint8_t *out, uint64_t h, uint64_t bound) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t lo[2] = {0, 0}, hi = 0;
+    if constexpr (DT == SZ_BF16) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            // exponents of elements 2k, 2k+1 in bytes 0 and 2
+            const uint32_t x = (w[k] >> 7) & 0x00FF00FFu;
+            lo[0] |= ((x & 0xFu) | ((x >> 12) & 0xF0u)) << (8 * k);
+            hi |= (((x >> 4) & 0xFu) | ((x >> 16) & 0xF0u)) << (8 * k);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t x = (w[j >> 2] >> (8 * (j & 3) + 2)) & 0x1Fu;
+            lo[j >> 3] |= (x & 0xFu) << (4 * (j & 7));
+            hi |= (x >> 4) << j;
+        }
+    }
+    constexpr int kHiBytes = (DT == SZ_BF16) ? 4 : 2;
+    if (valid == Geo<DT>::LE) {
+        if constexpr (DT == SZ_BF16) *reinterpret_cast<uint32_t *>(cd) = lo[0];
+        else *reinterpret_cast<uint2 *>(cd) = make_uint2(lo[0], lo[1]);
+        if (h + kHiBytes <= bound && (h & (kHiBytes - 1)) == 0) {
+            if constexpr (DT == SZ_BF16) *reinterpret_cast<uint32_t *>(out + h) = hi;
+            else *reinterpret_cast<uint16_t *>(out + h) = uint16_t(hi);
+            return;
+        }
+    } else {
+        store_bytes(cd, lo[0], lo[1], (valid + 1) / 2);
+    }
+    const int hbytes = (DT == SZ_BF16) ? (valid + 1) / 2 : (valid + 7) / 8;
+    for (int b = 0; b < hbytes; ++b)
+        if (h + b < bound) out[h + b] = uint8_t(hi >> (8 * b));
+}
+
 // One warp stores block blk raw (raw blocks allowed and its escapes would
 // fill at least raw_block_bytes): the low four bits of each exponent
 // overwrite the block's code nibbles, the remaining bits go to the escape
 // section at byte d (BF16: high nibbles, element j of the block in nibble j%2
 // of byte j/2; E5M2: bit 4 at bit j%8 of byte j/8), bytes at or past bound
-// not written.  Planes are as coded.  Rare by construction (data that the
-// codebook misses), so this reads its input again from global memory.
+// not written.  Planes are as coded.  The block's input is read again, with
+// G::kAhead loads per lane in flight for a full contiguous block.  Out of line:
+// inlined into the kernel it slowed the coded path by 1-2% (measured).
 template <int DT, bool PAGED>
-__device__ void raw_block(const uint8_t *in, const PageRef &pr, uint64_t n, uint64_t blk, const Layout &L,
+__device__ __noinline__ void raw_block(const uint8_t *in, const PageRef &pr, uint64_t n, uint64_t blk, const Layout &L,
                           uint8_t *out, uint64_t d, uint64_t bound) {
     using G = Geo<DT>;
+    constexpr int EB = Dt<DT>::kElemBytes;
     const int lane = threadIdx.x & 31;
     const uint64_t e_lane = blk * kBlock + uint64_t(lane) * G::LE;
     const bool paged = PAGED && pr.pages != nullptr;
     uint8_t *code = out + L.code + e_lane / 2;
+    // this lane's high bits of step it start at h0 + it * kHiStride
+    const uint64_t h0 = d + ((DT == SZ_BF16) ? uint64_t(lane) * G::LE / 2 : uint64_t(lane) * G::LE / 8);
+    constexpr uint32_t kHiStride = (DT == SZ_BF16) ? 32 * G::LE / 2 : 32 * G::LE / 8;
+    if (!paged && (blk + 1) * kBlock <= n) {
+        const uint8_t *src = in + e_lane * EB;
+        uint4 ring[G::kAhead + 1];
+#pragma unroll
+        for (int i = 0; i < G::kAhead; ++i) ring[i] = __ldcs(reinterpret_cast<const uint4 *>(src + i * 512));
+#pragma unroll
+        for (int it = 0; it < G::IT; ++it) {
+            if (it + G::kAhead < G::IT)
+                ring[(it + G::kAhead) % (G::kAhead + 1)] =
+                    __ldcs(reinterpret_cast<const uint4 *>(src + (it + G::kAhead) * 512));
+            raw_step<DT>(ring[it % (G::kAhead + 1)], G::LE, code + it * EStride<DT>::code, out,
+                         h0 + uint64_t(it) * kHiStride, bound);
+        }
+        return;
+    }
 #pragma unroll 1
     for (int it = 0; it < G::IT; ++it) {
         const int64_t left = int64_t(n) - int64_t(e_lane) - int64_t(it) * 32 * G::LE;
         const int valid = left <= 0 ? 0 : (left >= G::LE ? G::LE : int(left));
         if (valid <= 0) continue;
         const uint64_t e = e_lane + uint64_t(it) * 32 * G::LE;
-        const uint64_t off = paged ? elem_offset<Dt<DT>::kElemBytes>(pr, e) : e * Dt<DT>::kElemBytes;
+        const uint64_t off = paged ? elem_offset<EB>(pr, e) : e * EB;
         const uint4 v = off != kBadOffset ? load_step<DT>(in + off, valid) : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t lo[2] = {0, 0}, hi = 0;
-#pragma unroll
-        for (int j = 0; j < G::LE; ++j) {
-            uint32_t x;
-            if constexpr (DT == SZ_BF16) x = (w[j >> 1] >> (16 * (j & 1) + 7)) & 0xFFu;
-            else x = (w[j >> 2] >> (8 * (j & 3) + 2)) & 0x1Fu;
-            lo[j >> 3] |= (x & 0xFu) << (4 * (j & 7));
-            if constexpr (DT == SZ_BF16) hi |= (x >> 4) << (4 * j);
-            else hi |= (x >> 4) << j;
-        }
-        // code nibbles: the same bytes code_step wrote for this lane
-        store_bytes(code + it * EStride<DT>::code, lo[0], lo[1], (valid + 1) / 2);
-        // high bits: this lane's share of the block's raw_block_bytes
-        const uint32_t local = uint32_t(it) * 32 * G::LE + uint32_t(lane) * G::LE;  // within the block
-        const uint64_t h0 = d + ((DT == SZ_BF16) ? local / 2 : local / 8);
-        const int hbytes = (DT == SZ_BF16) ? (valid + 1) / 2 : (valid + 7) / 8;
-        for (int b = 0; b < hbytes; ++b)
-            if (h0 + b < bound) out[h0 + b] = uint8_t(hi >> (8 * b));
+        raw_step<DT>(v, valid, code + it * EStride<DT>::code, out, h0 + uint64_t(it) * kHiStride, bound);
     }
 }
 
@@ -639,15 +704,14 @@ __device__ __forceinline__ ChunkGeo chunk_geo(const EncodeParams<MAXB> &p, uint3
 }
 
 // One warp codes a chunk: planes and codes go out, escapes are staged in
-// esc[slot] (element order) with per-block offsets in blk_off[slot].  Between
-// blocks it calls between().  Returns the chunk's escape-section bytes, or
+// esc[slot] (element order) with per-block offsets in blk_off[slot].  Returns
+// the chunk's escape-section bytes, or
 // 0xFFFFFFFF if the plan does not fit the data (reported; nothing to finish).
 // With raw blocks allowed, bit k of *raw is set for each block k of the chunk
 // that is to be stored raw; it counts raw_block_bytes.
-template <int DT, int MAXB, bool PAGED, typename Between>
+template <int DT, int MAXB, bool PAGED>
 __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
-                               WarpShared &W, RingState &R, int &plan_tensor, bool *lost, uint32_t *raw,
-                               Between between) {
+                               WarpShared &W, RingState &R, int &plan_tensor, bool *lost, uint32_t *raw) {
     const int lane = threadIdx.x & 31;
     const uint8_t *in = p.in[g.t];
     uint8_t *out = p.out[g.t];
@@ -704,11 +768,13 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
             *lost = !ring_take(W, R, &st) || *lost;
             if (full) {
                 const uint32_t src = smem_u32(W.ring[st]) + uint32_t(lane) * 16;
+                // escapes that can no longer be staged are only counted (checked per unit)
+                const bool staged = base + blk_run < kWarpStage;
 #pragma unroll
                 for (int it = 0; it < QIT; ++it) {
                     const uint4 v = lds_u128(src + it * 512);
                     const EMask<DT> m = code_step<DT, true>(lut, v, G::LE, q, qq * QIT + it);
-                    rank_step<DT>(m, v, blk_run, put);
+                    rank_step<DT>(m, v, blk_run, put, staged);
                 }
             } else {
                 for (int it = qq * QIT; it < (qq + 1) * QIT; ++it) {
@@ -734,7 +800,6 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
             }
         }
         running += blk_run;
-        between();
     }
     __syncwarp();
     return running;
@@ -848,14 +913,13 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
     int plan_tensor = -1;
     Pending pend;
     pend.valid = false;
-    // finish the pending chunk once its look-back is done (blocking or not)
-    auto settle = [&](bool block) {
+    // finish the pending chunk (its look-back waits, bounded, until done)
+    auto settle = [&]() {
         if (!pend.valid) return;
         const ChunkGeo pg = chunk_geo<MAXB, LG>(p, pend.job);
-        if (lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, block)) {
-            finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W);
-            pend.valid = false;
-        }
+        lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, true);
+        finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W);
+        pend.valid = false;
     };
     // every warp claims chunks in launch order until none is left
     while (true) {
@@ -871,14 +935,13 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
         const int slot = pend.valid ? (pend.slot ^ 1) : 0;
         bool lost = false;
         uint32_t raw = 0;
-        const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost, &raw,
-                                                    [&]() { settle(false); });
+        const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost, &raw);
         if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
         if (total == 0xFFFFFFFFu) continue;  // plan rejected for this tensor
         unsigned long long *st = chunk_status(p, g.t);
         Lookback lb;
         lookback_start(lb, st, g.chunk, total, tag);
-        settle(true);  // at most one chunk waits for its offset
+        settle();  // at most one chunk waits for its offset
         // chunks that re-read their input (escape overflow, raw blocks) finish at once
         if (total > kWarpStage || raw != 0 || lookback_advance(lb, st, g.chunk, total, tag, false)) {
             lookback_advance(lb, st, g.chunk, total, tag, true);
@@ -891,7 +954,7 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
             pend.lb = lb;
         }
     }
-    settle(true);
+    settle();
     // The last CTA to retire leaves the counters ready for the next launch.
     __syncthreads();
     if (tid == 0) {
