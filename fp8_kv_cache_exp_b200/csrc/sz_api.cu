@@ -187,6 +187,7 @@ sz_status encode_common(sz_dtype dtype, int T, const sz_plan_t *d_plans, const v
     a.cap = out_cap;
     a.ctl = reinterpret_cast<uint32_t *>(ws);
     a.status = reinterpret_cast<unsigned long long *>(ws + w.status);
+    a.group = reinterpret_cast<unsigned long long *>(ws + w.group);
     a.totals = reinterpret_cast<unsigned long long *>(d_totals);
     a.reuse = reuse ? 1 : 0;
     a.paged = paged;

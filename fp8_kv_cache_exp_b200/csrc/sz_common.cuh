@@ -128,17 +128,25 @@ __host__ __device__ inline Layout stream_layout(int dtype, uint64_t n, uint64_t 
     return L;
 }
 
+// Encode's look-back works on two levels: one status word per chunk and one
+// per group of kLbGroup consecutive chunks of a tensor.
+constexpr int kLbGroupLog2 = 5;
+constexpr uint32_t kLbGroup = 1u << kLbGroupLog2;
+
 // Workspace partition: control block, per-tensor histograms and tickets
-// (plan), per-tile look-back status words (encode).
+// (plan), per-tile look-back status words and per-group words (encode; a
+// tensor's groups start at word (its first chunk >> kLbGroupLog2) + its index,
+// so total_tiles / kLbGroup + T + 1 words hold every launch's groups).
 struct WsLayout {
-    size_t hist, ticket, status, bytes;
+    size_t hist, ticket, status, group, bytes;
 };
 constexpr WsLayout ws_layout(int T, uint64_t total_tiles) {
     WsLayout w{};
     w.hist = kCtlWords * 4;
     w.ticket = w.hist + size_t(T) * 256 * 4;
     w.status = w.ticket + align256(size_t(T) * 4);
-    w.bytes = w.status + size_t(total_tiles) * 8;
+    w.group = w.status + align256(size_t(total_tiles) * 8);
+    w.bytes = w.group + (size_t(total_tiles >> kLbGroupLog2) + size_t(T) + 1) * 8;
     return w;
 }
 
@@ -179,6 +187,7 @@ template <int MAXB>
 struct EncodeParams {
     uint32_t *ctl;
     unsigned long long *status;  // one look-back word per global chunk
+    unsigned long long *group;   // one look-back word per group of kLbGroup chunks of a tensor
     const uint8_t *plans;
     unsigned long long *totals;  // per-tensor stream bytes out (may be null)
     int reuse;                   // plans give codebooks only: E and the total are found here

@@ -70,82 +70,143 @@ struct Geo {
     static constexpr int kAhead = 3;                        // steps of loads in flight
 };
 
-// Decoupled look-back of one chunk, run by one warp and resumable: the warp
-// publishes the chunk's aggregate, then sums its predecessors' published
-// values back to the nearest inclusive prefix.  Status word: epoch (30 bits)
-// << 34 | flag << 32 | value; words of earlier launches carry an older epoch
-// and read as "not published".  A round reads the 128 nearest unsummed
-// predecessors (lane l: positions 4l .. 4l + 3 behind the cursor, position 0
-// = nearest).  Every predecessor publishes its aggregate as soon as it has
+// Decoupled look-back of one chunk, run by one warp and resumable, on two
+// levels.  Status words (per chunk, and per group of kLbGroup consecutive
+// chunks of a tensor): epoch (30 bits) << 34 | flag << 32 | value; words of
+// earlier launches carry an older epoch and read as "not published".  A chunk
+// word holds the chunk's escape count (flag kFlagAgg) or its inclusive prefix
+// (kFlagInc); a group word holds the sum of its chunks (kFlagAgg) or the
+// inclusive prefix through its last chunk (kFlagInc).
+//   Phase 1: the chunk's own group -- the up to 31 predecessors in it, one per
+//   lane -- summed back to the nearest inclusive prefix.
+//   Phase 2: whole groups, 32 per round (1024 chunks), summed back to the
+//   nearest inclusive group word; the start of the tensor counts as an
+//   inclusive prefix of 0.  A needed group word not yet published is made by
+//   the warp itself from the group's chunk words, once they are all published.
+// Group words are also published by the last chunk of each group, right after
+// its own aggregate (if the group's other chunks are done) and with its own
+// inclusive prefix.  Every chunk publishes its aggregate as soon as it has
 // coded its chunk, without waiting on anything, so a look-back always ends;
-// the total wait is still bounded (SZ_ERR_TIMEOUT).  Measured variants: 512
-// predecessors per round made every encode slower; retrying a deferred
-// look-back between the blocks of the warp's next chunk (each try stalls the
-// warp for an L2 round trip) made the Llama-3-8B batch encode 4% and one
-// Qwen3-32B layer 8% slower than settling it once, after that chunk.
+// the total wait is still bounded (SZ_ERR_TIMEOUT).  When every chunk of a
+// launch finishes at about the same time (one chunk per warp), a one-level
+// look-back needs some j / 256 dependent rounds for chunk j; two levels need
+// two or three.  Measured variants: 512 predecessors per one-level round made
+// every encode slower; retrying a deferred look-back between the blocks of
+// the warp's next chunk (each try stalls the warp for an L2 round trip) made
+// the Llama-3-8B batch encode 4% and one Qwen3-32B layer 8% slower than
+// settling it once, after that chunk.
 struct Lookback {
-    int32_t j;      // nearest predecessor not yet summed
+    int32_t j;      // phase 1: nearest unsummed predecessor; phase 2: nearest unsummed group
     uint32_t excl;  // escapes summed so far
     uint32_t t0;    // low bits of the time a predecessor was first found unpublished
-    uint32_t flags; // kLbDone | kLbTimedOut | kLbWaiting
+    uint32_t flags; // kLbDone | kLbTimedOut | kLbWaiting | kLbGroups
 };
-constexpr uint32_t kLbDone = 1, kLbTimedOut = 2, kLbWaiting = 4;
-constexpr int kLookbackPerLane = 4;  // status words per lane per round
+constexpr uint32_t kLbDone = 1, kLbTimedOut = 2, kLbWaiting = 4, kLbGroups = 8;
 
-__device__ __forceinline__ void lookback_start(Lookback &lb, unsigned long long *st, uint32_t chunk,
-                                               uint32_t agg, unsigned long long tag) {
-    lb.j = int32_t(chunk) - 1;
+// A tensor's look-back words: its chunk words, its group words, its chunk count.
+struct LbWords {
+    unsigned long long *st, *gs;
+    uint32_t nchunks;
+};
+
+// Flag (0: not published in this launch) and value of a status word.
+__device__ __forceinline__ uint32_t lb_flag(unsigned long long w, unsigned long long tag) {
+    return ((w >> 34) == (tag >> 34)) ? uint32_t(w >> 32) & 3u : 0u;
+}
+
+// Publish word w (flag f) for group g unless it already holds as much (an
+// inclusive prefix beats an aggregate); one compare-and-swap, losing a race
+// to another publisher is fine (both words are true).
+__device__ __forceinline__ void publish_group(const LbWords &c, uint32_t g, unsigned long long w,
+                                              unsigned long long tag) {
+    const unsigned long long cur = ld_relaxed_u64(c.gs + g);
+    if (lb_flag(cur, tag) < lb_flag(w, tag)) atomicCAS(c.gs + g, cur, w);
+}
+
+// Try to make group g's word from its chunk words (one round, warp-wide):
+// true if it is published now.
+__device__ bool make_group(const LbWords &c, uint32_t g, unsigned long long tag) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t k = (g << kLbGroupLog2) + uint32_t(lane);
+    uint32_t f = 2, v = 0;  // chunks past the tensor's end: nothing to add
+    if (k < c.nchunks) {
+        const unsigned long long w = ld_relaxed_u64(c.st + k);
+        f = lb_flag(w, tag);
+        v = uint32_t(w);
+    }
+    if (!__all_sync(0xffffffffu, f != 0)) return false;
+    // the last inclusive prefix among the group's chunks, then the aggregates after it
+    const uint32_t inc = __ballot_sync(0xffffffffu, k < c.nchunks && f == 2);
+    const int L = inc ? 31 - __clz(inc) : -1;
+    const uint32_t sum = __reduce_add_sync(0xffffffffu, (lane >= L && k < c.nchunks) ? v : 0u);
+    if (lane == 0)
+        publish_group(c, g, tag | (L >= 0 ? kFlagInc : kFlagAgg) | sum, tag);
+    return true;
+}
+
+__device__ __forceinline__ void lookback_start(Lookback &lb, const LbWords &c, uint32_t chunk, uint32_t agg,
+                                               unsigned long long tag) {
+    const int lane = threadIdx.x & 31;
     lb.excl = 0;
     lb.t0 = 0;
     lb.flags = chunk == 0 ? kLbDone : 0u;
-    if ((threadIdx.x & 31) == 0) st_relaxed_u64(st + chunk, tag | (chunk == 0 ? kFlagInc : kFlagAgg) | agg);
+    lb.j = int32_t(chunk) - 1;
+    if (chunk != 0 && (chunk & (kLbGroup - 1)) == 0) {  // first chunk of its group: no phase 1
+        lb.flags |= kLbGroups;
+        lb.j = int32_t(chunk >> kLbGroupLog2) - 1;
+    }
+    if (lane == 0) st_relaxed_u64(c.st + chunk, tag | (chunk == 0 ? kFlagInc : kFlagAgg) | agg);
+    // the last chunk of a group publishes the group's word if the others are done
+    if ((chunk & (kLbGroup - 1)) == kLbGroup - 1 || chunk + 1 == c.nchunks) {
+        __syncwarp();
+        make_group(c, chunk >> kLbGroupLog2, tag);
+    }
 }
 
-// Sum published predecessors of chunk (status words st, own count agg); with
-// `block`, wait until done.  Returns true once the chunk's offset is known.
-__device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t chunk, uint32_t agg,
+// Sum published predecessors of chunk (own count agg); with `block`, wait
+// until done.  Returns true once the chunk's offset is known.
+__device__ bool lookback_advance(Lookback &lb, const LbWords &c, uint32_t chunk, uint32_t agg,
                                  unsigned long long tag, bool block) {
     const int lane = threadIdx.x & 31;
     uint32_t backoff = 32;
     while (!(lb.flags & kLbDone)) {
-        constexpr int w = kLookbackPerLane;
-        unsigned long long word[w];
-#pragma unroll
-        for (int q = 0; q < w; ++q) {
-            const int32_t idx = lb.j - w * lane - q;
-            word[q] = idx >= 0 ? ld_relaxed_u64(st + idx) : 0ull;
+        const bool groups = (lb.flags & kLbGroups) != 0;
+        // phase 1: predecessor lb.j - lane of the own group; phase 2: group lb.j - lane
+        const int32_t first = groups ? 0 : int32_t(chunk & ~(kLbGroup - 1));
+        const int32_t idx = lb.j - lane;
+        uint32_t f = 2, v = 0;  // before the group's (phase 1) or tensor's (phase 2) start: inclusive 0
+        if (idx >= first) {
+            const unsigned long long w = ld_relaxed_u64((groups ? c.gs : c.st) + idx);
+            f = lb_flag(w, tag);
+            v = uint32_t(w);
+        } else if (!groups) {
+            f = 3;  // phase 1 past the own group's start: not needed, ends the phase
         }
-        // this lane's positions up to and including its nearest inclusive prefix
-        // (all w of them if it has none): their sum and whether all are published
-        int my_inc = w;
-        uint32_t sum = 0;
-        bool ready = true;
-#pragma unroll
-        for (int q = 0; q < w; ++q) {
-            if (my_inc == w) {
-                const int32_t idx = lb.j - w * lane - q;
-                // before chunk 0: a virtual inclusive prefix of 0
-                const uint32_t f = idx < 0 ? 2u
-                                           : (((word[q] >> 34) == (tag >> 34)) ? uint32_t(word[q] >> 32) & 3u : 0u);
-                sum += idx < 0 ? 0u : uint32_t(word[q]);
-                ready = ready && f != 0;
-                if (f == 2) my_inc = q;
-            }
-        }
-        const uint32_t inc_lanes = __ballot_sync(0xffffffffu, my_inc < w);
-        const int L = inc_lanes ? __ffs(inc_lanes) - 1 : 32;
-        if (lane > L) {  // past the nearest inclusive prefix: not needed
-            sum = 0;
-            ready = true;
-        }
-        if (__all_sync(0xffffffffu, ready)) {
-            lb.excl += __reduce_add_sync(0xffffffffu, sum);
-            if (L < 32) {
+        const uint32_t stop = __ballot_sync(0xffffffffu, f >= 2);
+        const int L = stop ? __ffs(stop) - 1 : 32;  // nearest inclusive prefix (or phase end)
+        const bool need = lane < L || (lane == L && f == 2);
+        if (__all_sync(0xffffffffu, !need || f != 0)) {
+            lb.excl += __reduce_add_sync(0xffffffffu, need ? v : 0u);
+            if (L < 32 && __shfl_sync(0xffffffffu, f, L) == 2) {
                 lb.flags |= kLbDone;
                 break;
             }
-            lb.j -= 32 * w;
+            if (groups) {
+                lb.j -= 32;
+            } else {  // own group summed: continue with the groups before it
+                lb.flags |= kLbGroups;
+                lb.j = int32_t(chunk >> kLbGroupLog2) - 1;
+                if (lb.j < 0) {
+                    lb.flags |= kLbDone;
+                    break;
+                }
+            }
             continue;
+        }
+        if (groups) {
+            // make the nearest missing group word, then try again at once
+            const uint32_t miss = __ballot_sync(0xffffffffu, need && f == 0);
+            if (make_group(c, uint32_t(lb.j - (__ffs(miss) - 1)), tag)) continue;
         }
         const uint32_t now = __shfl_sync(0xffffffffu, uint32_t(global_ns()), 0);
         if (!(lb.flags & kLbWaiting)) {
@@ -159,7 +220,13 @@ __device__ bool lookback_advance(Lookback &lb, unsigned long long *st, uint32_t 
         __nanosleep(backoff);
         if (backoff < 256) backoff <<= 1;
     }
-    if (chunk != 0 && lane == 0) st_relaxed_u64(st + chunk, tag | kFlagInc | (lb.excl + agg));
+    if (chunk != 0 && lane == 0) {
+        const unsigned long long w = tag | kFlagInc | (lb.excl + agg);
+        st_relaxed_u64(c.st + chunk, w);
+        // the last chunk of a group: its inclusive prefix is the group's
+        if ((chunk & (kLbGroup - 1)) == kLbGroup - 1 || chunk + 1 == c.nchunks)
+            publish_group(c, chunk >> kLbGroupLog2, w, tag);
+    }
     return true;
 }
 
@@ -887,9 +954,14 @@ struct Pending {
     Lookback lb;
 };
 
+// Tensor t's look-back words.
 template <int MAXB>
-__device__ __forceinline__ unsigned long long *chunk_status(const EncodeParams<MAXB> &p, int t) {
-    return p.status + p.chunk_begin[t];
+__device__ __forceinline__ LbWords lb_words(const EncodeParams<MAXB> &p, int t) {
+    LbWords c;
+    c.st = p.status + p.chunk_begin[t];
+    c.gs = p.group + (p.chunk_begin[t] >> kLbGroupLog2) + uint32_t(t);
+    c.nchunks = p.chunk_begin[t + 1] - p.chunk_begin[t];
+    return c;
 }
 
 template <int DT, int MAXB, bool PAGED, int LG>
@@ -917,7 +989,7 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
     auto settle = [&]() {
         if (!pend.valid) return;
         const ChunkGeo pg = chunk_geo<MAXB, LG>(p, pend.job);
-        lookback_advance(pend.lb, chunk_status(p, pg.t), pg.chunk, pend.total, tag, true);
+        lookback_advance(pend.lb, lb_words(p, pg.t), pg.chunk, pend.total, tag, true);
         finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W);
         pend.valid = false;
     };
@@ -938,7 +1010,7 @@ __global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const
         const uint32_t total = code_chunk<DT, MAXB, PAGED>(p, job, g, slot, W, R, plan_tensor, &lost, &raw);
         if (lost && lane == 0) set_error(p.ctl, SZ_ERR_TIMEOUT, job);
         if (total == 0xFFFFFFFFu) continue;  // plan rejected for this tensor
-        unsigned long long *st = chunk_status(p, g.t);
+        const LbWords st = lb_words(p, g.t);
         Lookback lb;
         lookback_start(lb, st, g.chunk, total, tag);
         settle();  // at most one chunk waits for its offset
@@ -982,6 +1054,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     EncodeParams<MAXB> p;
     p.ctl = a.ctl;
     p.status = a.status;
+    p.group = a.group;
     p.plans = a.plans;
     p.totals = a.totals;
     p.reuse = a.reuse;

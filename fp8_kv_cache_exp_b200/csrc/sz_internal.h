@@ -27,6 +27,7 @@ struct EncodeArgs {
     const size_t *cap;
     uint32_t *ctl;
     unsigned long long *status;
+    unsigned long long *group;
     unsigned long long *totals;  // may be null
     int reuse;                   // codebook reuse: plans give codebooks only
     const sz_paged_t *paged;     // T input page descriptors, or null (contiguous inputs)

@@ -21,10 +21,11 @@ namespace {
 
 // Largest tensor this entry point accepts, and the scratch it needs: the
 // workspace of one tensor of that size (control block, histogram, ticket, one
-// look-back status word per 4096-element tile) -- 263,680 bytes.
+// look-back status word per 4096-element tile and one per 32 of them) --
+// 271,888 bytes.
 constexpr uint64_t kNoAllocMaxTiles = SZ_NOALLOC_MAX_ELEMS / sz::kBlock;
 constexpr size_t kNoAllocScratchBytes = sz::ws_layout(1, kNoAllocMaxTiles).bytes;
-static_assert(kNoAllocScratchBytes == 263680, "the header states the scratch size");
+static_assert(kNoAllocScratchBytes == 271888, "the header states the scratch size");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -298,7 +298,7 @@ sz_status sz_last_device_status(void *d_ws, cudaStream_t stream);
  * example an engine that reserves all of the GPU's memory for its KV pool at
  * start-up and hands the codec only the tensor, the destination buffer and a
  * stream.  The call runs the same kernel as sz_encode on a scratch area held
- * by the library: a static device array of 263,680 bytes (the workspace of
+ * by the library: a static device array of 271,888 bytes (the workspace of
  * one tensor of SZ_NOALLOC_MAX_ELEMS elements) that every GPU which loads the
  * library keeps until the process exits.  It calls no cudaMalloc, cudaFree or other
  * allocating routine; it enqueues a memset of the scratch it uses, the encode

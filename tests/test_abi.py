@@ -62,9 +62,12 @@ def test_host_sizes_match_oracle(lib, dtype):
 
 def test_workspace_sizes(lib):
     import fp8_kv_cache_exp_b200 as sz
+    # control block, histograms, tickets, one look-back word per 4096-element
+    # block, then one per 32 blocks plus one per tensor and one more
     one = sz.sz_workspace_bytes(0, 8388608)
-    assert one == 256 + 1024 + 256 + 8 * 2048
-    assert sz.sz_workspace_bytes_batched(0, [8388608] * 64) == 256 + 64 * 1024 + 256 + 8 * 2048 * 64
+    assert one == 256 + 1024 + 256 + 8 * 2048 + 8 * (2048 // 32 + 1 + 1)
+    assert sz.sz_workspace_bytes_batched(0, [8388608] * 64) == \
+        256 + 64 * 1024 + 256 + 8 * 2048 * 64 + 8 * (2048 * 64 // 32 + 64 + 1)
     assert sz.sz_workspace_bytes_batched(0, [1] * 257) == 0
 
 
