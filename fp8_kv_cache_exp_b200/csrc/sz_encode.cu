@@ -35,13 +35,15 @@ namespace sz {
 
 namespace {
 
-// Persistent CTAs of 8 independent warps: 3 per SM at 80 registers (BF16), 2
-// per SM at 128 registers (E5M2 does more work per loaded byte and runs faster
-// with more registers).  Measured against one CTA of 24 (16) warps per SM:
-// the same on large batches, slower on one Qwen3-32B layer (0.70 against
-// 0.76 of the HBM peak).
-constexpr int NT = kTileThreads;
-constexpr int NW = NT / 32;
+// Persistent CTAs of independent warps, 24 per SM at 80 registers: 3 CTAs of
+// 8 warps for BF16, 2 CTAs of 12 for E5M2 (measured best among 2 x 8 warps at
+// 128 registers, 2 x 10 at 96, 3 x 7 at 96 and 2 x 12 at 80, with the E5M2
+// step loop rolled).  One CTA of 24 warps per SM was the same on large batches
+// and slower on one Qwen3-32B layer (0.70 against 0.76 of the HBM peak).
+template <int DT>
+constexpr int enc_threads() { return DT == SZ_BF16 ? kTileThreads : 384; }
+template <int DT>
+constexpr int enc_ctas_per_sm() { return DT == SZ_BF16 ? 3 : 2; }
 constexpr int kChunkBlocks = kMaxChunkBlocks;         // a warp's unit of work: up to 8 consecutive blocks
 constexpr uint32_t kWarpStage = 1024;                 // staged escape bytes per chunk (two chunks)
 constexpr int kRing = 3;                              // input-unit stages per warp
@@ -975,7 +977,7 @@ __device__ __forceinline__ LbWords lb_words(const EncodeParams<MAXB> &p, int t) 
 }
 
 template <int DT, int MAXB, bool PAGED, int LG>
-__global__ void __launch_bounds__(NT, DT == SZ_BF16 ? 3 : 2) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
+__global__ void __launch_bounds__(enc_threads<DT>(), enc_ctas_per_sm<DT>()) encode_kernel(const __grid_constant__ EncodeParams<MAXB> p) {
     extern __shared__ __align__(128) uint8_t s_raw[];
     WarpShared *s_warp = reinterpret_cast<WarpShared *>(s_raw);
     __shared__ uint32_t s_epoch;
@@ -1054,6 +1056,7 @@ sz_status launch_encode_t(const EncodeArgs &a, cudaStream_t stream) {
     // Full-size chunks (large batches) run an instantiation with the chunk size
     // fixed at compile time; shorter chunks read it from the launch.  Both have
     // the same launch bounds and shared memory.
+    constexpr int NT = enc_threads<DT>(), NW = NT / 32;
     auto kern_full = encode_kernel<DT, MAXB, PAGED, kMaxChunkLog2>;
     auto kern_any = encode_kernel<DT, MAXB, PAGED, -1>;
     const size_t smem = sizeof(WarpShared) * NW;
