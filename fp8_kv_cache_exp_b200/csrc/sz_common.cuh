@@ -219,17 +219,16 @@ struct DecodeParams {
     PageRef pg[MAXB];                // output pages
 };
 
-// Blocks per chunk for a launch: the largest power of two (<= kMaxChunkBlocks)
-// that still gives at least one chunk per two resident warps.  Every chunk
-// costs a claim, a look-back and a ring restart, so chunks stay as long as the
-// launch allows: a large batch keeps 8-block chunks, one layer's K and V
-// (4096 BF16 or 8192 E5M2 blocks) gets 2- or 4-block chunks and still spreads
-// over every SM (measured best for both; 1-block chunks for one Llama-3-8B
-// layer took 25% longer).
+// Blocks per chunk for a launch.  Every chunk costs a claim, a look-back and a
+// ring restart, so chunks are as long as the launch allows: 8 blocks if that
+// still gives at least one chunk per two resident warps, else 2 blocks -- 1 if
+// even that leaves fewer chunks than half the resident warps.  Measured: the
+// Llama-3-8B and E5M2 batches and a cold Qwen3-32B layer are fastest in
+// 8-block chunks; one Llama-3-8B or E5M2 layer (4096 or 8192 blocks) in 2-block
+// chunks (1-block: 13% slower for Llama-3-8B; 4-block: 8% slower for E5M2).
 inline int pick_chunk_log2(uint64_t total_blocks, uint64_t resident_warps) {
-    int lg = kMaxChunkLog2;
-    while (lg > 0 && (total_blocks >> lg) < resident_warps / 2) --lg;
-    return lg;
+    if ((total_blocks >> kMaxChunkLog2) >= resident_warps / 2) return kMaxChunkLog2;
+    return (total_blocks >> 1) >= resident_warps / 2 ? 1 : 0;
 }
 
 // ------------------------------------------------ programmatic dependent launch

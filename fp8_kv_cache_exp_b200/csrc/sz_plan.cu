@@ -60,9 +60,13 @@ __device__ __forceinline__ void count_vec(uint32_t col, uint32_t inc, uint4 v) {
             red_shared_add(col + ((w[k] >> 7) & 0xFFu) * kRowBytes, inc);
             red_shared_add(col + ((w[k] >> 23) & 0xFFu) * kRowBytes, inc);
         } else {
-            // four elements per word: exponent bits 2..6 of each byte
+            // four elements per word: exponent bits 2..6 of each byte, all four
+            // extracted by one shift and mask, then each moved to byte 0 by a
+            // byte permute (about 2.5 integer ops per element instead of 3)
+            const uint32_t x = (w[k] >> 2) & 0x1F1F1F1Fu;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) red_shared_add(col + ((w[k] >> (8 * b + 2)) & 0x1Fu) * kRowBytes, inc);
+            for (int b = 0; b < 4; ++b)
+                red_shared_add(col + __byte_perm(x, 0u, 0x4440u + uint32_t(b)) * kRowBytes, inc);
         }
     }
 }
