@@ -632,8 +632,13 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
         for (int k = 0; k < G::kAhead; ++k) issued |= feed.issue_next(W);
 
         WarpStream ws;
+        // BF16 reads the block's offsets-table entries (inside the buffer: the
+        // host checked its size) beside the header, not after it (per-layer
+        // decode 1.4% faster; E5M2 0.8% slower, so it keeps the other order)
+        BlockEsc be;
+        if constexpr (DT == SZ_BF16) be = load_offsets(p.comp[t], blk);
         warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
-        BlockEsc be = load_offsets(p.comp[t], blk);
+        if constexpr (DT != SZ_BF16) be = load_offsets(p.comp[t], blk);
         uint32_t esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
         uint32_t v = 0;  // units consumed
 
@@ -754,8 +759,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                 esc_reg = esc_n;
             } else {
                 t = t_n;
+                if constexpr (DT == SZ_BF16) be = load_offsets(p.comp[t], blk_n);
                 warp_open_stream<DT, MAXB>(p, t, W.tab, ws);
-                be = load_offsets(p.comp[t], blk_n);
+                if constexpr (DT != SZ_BF16) be = load_offsets(p.comp[t], blk_n);
                 esc_reg = ws.ok ? load_escape_reg(p.comp[t], ws, be) : 0u;
             }
             blk = blk_n;

@@ -894,11 +894,13 @@ __device__ uint32_t code_chunk(const EncodeParams<MAXB> &p, uint32_t job, const 
 // escapes (from the stage, or re-coded from the input when they overflowed
 // it or the chunk has raw blocks -- the warp's code table is then still the
 // chunk's), and the stream frame if it is the tensor's last chunk.
+// hdr_here: the warp's shared copy of the plan (W.hdr) is this chunk's tensor's,
+// so it is read instead of the plan in global memory.
 template <int DT, int MAXB, bool PAGED>
 __device__ void finish_chunk(const EncodeParams<MAXB> &p, uint32_t job, const ChunkGeo &g, int slot,
-                             uint32_t total, uint32_t raw, const Lookback &lb, WarpShared &W) {
+                             uint32_t total, uint32_t raw, const Lookback &lb, WarpShared &W, bool hdr_here) {
     const int lane = threadIdx.x & 31;
-    const Header H = load_header(p.plans + 64 * size_t(g.t));
+    const Header H = load_header(hdr_here ? reinterpret_cast<const uint8_t *>(W.hdr) : p.plans + 64 * size_t(g.t));
     const bool reuse = p.reuse != 0;
     // the plan's E counts every escape; raw blocks store fewer bytes, so with
     // raw blocks allowed E is known only at the end, as with a reused codebook
@@ -1008,7 +1010,7 @@ __global__ void __launch_bounds__(enc_threads<DT>(), enc_ctas_per_sm<DT>()) enco
         if (!pend.valid) return;
         const ChunkGeo pg = chunk_geo<MAXB, LG>(p, pend.job);
         lookback_advance(pend.lb, lb_words(p, pg.t), pg.chunk, pend.total, tag, true);
-        finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W);
+        finish_chunk<DT, MAXB, PAGED>(p, pend.job, pg, pend.slot, pend.total, 0u, pend.lb, W, pg.t == plan_tensor);
         pend.valid = false;
     };
     // every warp claims chunks in launch order until none is left
@@ -1035,7 +1037,7 @@ __global__ void __launch_bounds__(enc_threads<DT>(), enc_ctas_per_sm<DT>()) enco
         // chunks that re-read their input (escape overflow, raw blocks) finish at once
         if (total > kWarpStage || raw != 0 || lookback_advance(lb, st, g.chunk, total, tag, false)) {
             lookback_advance(lb, st, g.chunk, total, tag, true);
-            finish_chunk<DT, MAXB, PAGED>(p, job, g, slot, total, raw, lb, W);
+            finish_chunk<DT, MAXB, PAGED>(p, job, g, slot, total, raw, lb, W, g.t == plan_tensor);
         } else {
             pend.valid = true;
             pend.job = job;
