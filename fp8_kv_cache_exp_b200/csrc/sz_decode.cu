@@ -330,30 +330,57 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
             patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
         }
     } else {
-        // Escapes first.  With at most one escape per lane (the usual case) its
-        // exponent takes the place of code 15's byte in this lane's table, so the
-        // lookups below produce it directly; otherwise (general) the escapes are
-        // patched in afterwards.
-        const uint64_t m = uint64_t(escape_nibbles(f.c0)) | (uint64_t(escape_nibbles(f.c1)) << 32);
-        const uint32_t c = __popcll(m);
+        // Escapes first.  With one escape in a lane (the usual case) its exponent
+        // takes the place of code 15's byte in this lane's table, so the lookups
+        // below produce it directly.  With two, both read that byte; the second
+        // (in element order) is then corrected by the difference of the two
+        // exponents, which never carries out of its byte.  Ranks come from the
+        // ballots of "has one" and "has two".  Three or more (rare) take the
+        // general path.  The escape bytes held in esc_reg were checked once for
+        // the block (below 32); one read from global memory is checked here.
+        const uint32_t n0 = escape_nibbles(f.c0), n1 = escape_nibbles(f.c1);
+        const uint64_t m = uint64_t(n0) | (uint64_t(n1) << 32);
+        const uint32_t c = __popc(n0) + __popc(n1);
         const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
         uint32_t xt3 = xt[3];
         bool general = false;
+        uint32_t two = 0, fix_k = 0, fix_add = 0;
         if (any != 0) {
-            if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+            two = __ballot_sync(0xffffffffu, c > 1);
+            if (two == 0 || __ballot_sync(0xffffffffu, c > 2) == 0) {
                 const uint32_t lane = threadIdx.x & 31;
-                const uint32_t r = running + __popc(any & ((1u << lane) - 1u));
+                const uint32_t lt = (1u << lane) - 1u;
+                const uint32_t r = running + __popc(any & lt) + (two ? __popc(two & lt) : 0u);
                 const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
                 if (c) {
-                    uint32_t e = 0;
-                    if (r < cnt) e = (r < 32) ? v : uint32_t(esc_g[r]);
-                    else bad = true;
-                    if (e >= 32u) bad = true;
+                    uint32_t e = v;
+                    if (r >= 32) {
+                        e = r < cnt ? uint32_t(esc_g[r]) : 0u;
+                        bad = bad || e >= 32u;
+                    }
                     xt3 = (xt3 & 0x00FFFFFFu) | ((e & 31u) << 26);  // table byte 15 = exponent x 4 (< 128)
+                    fix_add = e;
                 }
-                running += __popc(any);
+                if (two) {
+                    const uint32_t v2 = __shfl_sync(0xffffffffu, esc_reg, (r + 1) & 31);
+                    if (c == 2) {
+                        uint32_t e2 = v2;
+                        if (r + 1 >= 32) {
+                            e2 = r + 1 < cnt ? uint32_t(esc_g[r + 1]) : 0u;
+                            bad = bad || e2 >= 32u;
+                        }
+                        // the second escape: the highest flagged nibble
+                        const uint32_t j = n1 ? 8u + ((31u - __clz(n1)) >> 2) : (31u - __clz(n0)) >> 2;
+                        fix_k = j >> 2;
+                        fix_add = ((e2 & 31u) - (fix_add & 31u)) << (2 + 8 * (j & 3));
+                    } else {
+                        fix_add = 0;
+                    }
+                }
+                running += __popc(any) + __popc(two);
             } else {
                 general = true;
+                two = 0;
             }
         }
         // four codes per word select their exponents from the register table:
@@ -375,6 +402,10 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
             const uint32_t mn = prmt(ev, 0u, 0x4440u + uint32_t(k)) * 0x1001u +
                                 prmt(od, 0u, 0x4440u + uint32_t(k)) * 0x40040u;
             o[k] = ((sg & 0x80808080u) | e_hi) | ((mn & 0x03030303u) | e_lo);
+        }
+        if (two) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] += (fix_k == uint32_t(k)) ? fix_add : 0u;
         }
         if (general) patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
     }
@@ -667,7 +698,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
                     qoff = elem_offset<EB>(p.pg[t], uint64_t(blk) * kBlock + uint64_t(lane) * G::kUnitElems);
             }
             uint32_t running = 0;
-            bool bad = false, timed_out = false;
+            // E5M2: the block's first 32 escape bytes, held in esc_reg, must be exponents
+            bool bad = DT == SZ_FP8_E5M2 && __any_sync(0xffffffffu, esc_reg >= 32u), timed_out = false;
             for (int q = 0; q < G::kUnits; ++q, ++v) {
                 if (q == G::kResolveQ) {
                     blk_n = claim_resolve<MAXB>(p, t_n, pend);

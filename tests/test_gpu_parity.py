@@ -235,3 +235,30 @@ def test_calls_capture_into_a_cuda_graph():
                 assert tot == ref.size and np.array_equal(out[:tot].cpu().numpy(), ref)
                 assert np.array_equal(dec.view(torch.uint8).cpu().numpy(), r)
         del graph
+
+
+@pytest.mark.parametrize("per_lane", [1, 2, 3], ids=["one", "two", "three"])
+@pytest.mark.parametrize("dtype", [0, 1], ids=["bf16", "e5m2"])
+def test_escapes_per_lane_step(dtype, per_lane):
+    """Every lane's share of every decode step (8 BF16 or 16 E5M2 consecutive
+    elements) holds exactly `per_lane` escapes, at random places, so that each
+    block has hundreds of escapes (ranks far past the 32 a warp holds in
+    registers) and every step takes the one-, two- or three-or-more-escape path.
+    Fifteen common exponents fill the rest; the escapes take rare ones."""
+    rng = np.random.default_rng(31 * per_lane + dtype)
+    le = 8 if dtype == 0 else 16
+    n = 4096 * 5 + 3 * le + 5  # whole blocks, then a ragged tail
+    common = np.arange(100, 115) if dtype == 0 else np.arange(5, 20)
+    # many rare values, each less frequent than any common one, so that all escape
+    rare = np.arange(40, 72) if dtype == 0 else np.setdiff1d(np.arange(32), common)
+    e = rng.choice(common, n)
+    for g in range(0, n - le + 1, le):
+        pos = rng.choice(le, per_lane, replace=False)
+        e[g + pos] = rng.choice(rare, per_lane)
+    if dtype == 0:
+        w = (rng.integers(0, 2, n) << 15) | (e << 7) | rng.integers(0, 128, n)
+        raw = w.astype(np.uint16).view(np.uint8)
+    else:
+        w = (rng.integers(0, 2, n) << 7) | (e << 2) | rng.integers(0, 4, n)
+        raw = w.astype(np.uint8)
+    check_parity(dtype, raw)
