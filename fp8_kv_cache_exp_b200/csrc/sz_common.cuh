@@ -447,6 +447,13 @@ __device__ __forceinline__ uint32_t warp_exclusive_prefix(uint32_t c, uint32_t *
     return x - c;
 }
 
+// Lanes below this one (bit i set for lane i < this lane).
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
 // Nibble flags of the escape code 15 among 8 packed 4-bit codes: bit 4j set
 // when code j is 15.
 __device__ __forceinline__ uint32_t escape_nibbles(uint32_t cw) {

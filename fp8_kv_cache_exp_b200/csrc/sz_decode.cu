@@ -332,25 +332,36 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
     } else {
         // Escapes first.  With one escape in a lane (the usual case) its exponent
         // takes the place of code 15's byte in this lane's table, so the lookups
-        // below produce it directly.  With two, both read that byte; the second
-        // (in element order) is then corrected by the difference of the two
-        // exponents, which never carries out of its byte.  Ranks come from the
-        // ballots of "has one" and "has two".  Three or more (rare) take the
-        // general path.  The escape bytes held in esc_reg were checked once for
-        // the block (below 32); one read from global memory is checked here.
+        // below produce it directly.  The common step -- at most one escape per
+        // lane, in a block with at most 32 -- runs straight through: the rank
+        // counts the lanes before this one that have an escape, the exponent
+        // comes from esc_reg (masked to 5 bits for the block), and a lane
+        // without an escape loads some other lane's byte into a slot it never
+        // selects.  Otherwise: with two escapes in a lane both read that byte
+        // and the second (in element order) is corrected by the difference of
+        // the two exponents, which never carries out of its byte; ranks come
+        // from the ballots of "has one" and "has two".  Three or more (rare)
+        // take the general path.  Escapes read from global memory (rank 32 and
+        // up) are checked here; a stream with more escapes than the block's
+        // count gives a count mismatch at the block's end.
         const uint32_t n0 = escape_nibbles(f.c0), n1 = escape_nibbles(f.c1);
         const uint64_t m = uint64_t(n0) | (uint64_t(n1) << 32);
-        const uint32_t c = __popc(n0) + __popc(n1);
-        const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+        const uint32_t fl = n0 | (n1 << 1);  // one bit per escaped element
+        const uint32_t any = __ballot_sync(0xffffffffu, fl != 0u);
+        const uint32_t multi = __ballot_sync(0xffffffffu, (fl & (fl - 1u)) != 0u);
         uint32_t xt3 = xt[3];
         bool general = false;
-        uint32_t two = 0, fix_k = 0, fix_add = 0;
-        if (any != 0) {
-            two = __ballot_sync(0xffffffffu, c > 1);
-            if (two == 0 || __ballot_sync(0xffffffffu, c > 2) == 0) {
-                const uint32_t lane = threadIdx.x & 31;
-                const uint32_t lt = (1u << lane) - 1u;
-                const uint32_t r = running + __popc(any & lt) + (two ? __popc(two & lt) : 0u);
+        uint32_t two = 0, fix_k = 0, fix_add = 0, c = 0;
+        if (multi == 0u && cnt <= 32u) {
+            const uint32_t r = running + __popc(any & lanemask_lt());
+            xt3 += __shfl_sync(0xffffffffu, esc_reg, r) << 26;  // source lane r mod 32
+            running += __popc(any);
+        } else {
+            c = __popc(n0) + __popc(n1);
+            two = multi;
+            if (__ballot_sync(0xffffffffu, c > 2) == 0) {
+                const uint32_t lt = lanemask_lt();
+                const uint32_t r = running + __popc(any & lt) + __popc(two & lt);
                 const uint32_t v = __shfl_sync(0xffffffffu, esc_reg, r & 31);
                 if (c) {
                     uint32_t e = v;
@@ -403,11 +414,14 @@ __device__ __forceinline__ void decode_step(const DFrag &f, uint32_t tab, const 
                                 prmt(od, 0u, 0x4440u + uint32_t(k)) * 0x40040u;
             o[k] = ((sg & 0x80808080u) | e_hi) | ((mn & 0x03030303u) | e_lo);
         }
-        if (two) {
+        if (two != 0u || general) {
+            if (two) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] += (fix_k == uint32_t(k)) ? fix_add : 0u;
+                for (int k = 0; k < 4; ++k) o[k] += (fix_k == uint32_t(k)) ? fix_add : 0u;
+            } else {
+                patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
+            }
         }
-        if (general) patch_escapes<DT>(o, m, c, running, esc_reg, esc_g, cnt, bad);
     }
     if (CHECKED && !store) {
         // an output page outside the pool: nothing is written
@@ -700,6 +714,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams<MAXB> &p) {
             uint32_t running = 0;
             // E5M2: the block's first 32 escape bytes, held in esc_reg, must be exponents
             bool bad = DT == SZ_FP8_E5M2 && __any_sync(0xffffffffu, esc_reg >= 32u), timed_out = false;
+            if (DT == SZ_FP8_E5M2) esc_reg &= 31u;
             for (int q = 0; q < G::kUnits; ++q, ++v) {
                 if (q == G::kResolveQ) {
                     blk_n = claim_resolve<MAXB>(p, t_n, pend);

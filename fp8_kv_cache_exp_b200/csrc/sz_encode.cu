@@ -431,15 +431,20 @@ __device__ __forceinline__ EMask<DT> code_step(uint32_t lut, uint4 v, int valid,
                 const uint32_t c = lds_u8(prmt(w[k], lut, 0x7650u + uint32_t(b)));
                 cw[k >> 1] += c << (4 * (4 * (k & 1) + b));
             }
-            if (STORE) {
-                // gathers by multiplication (no two partial products share a
-                // bit): the four sign bits to bits 28-31, the four 2-bit
-                // mantissas to bits 24-31; then to their place in the planes
-                const uint32_t sg = (w[k] & 0x80808080u) * 0x00204081u;
-                const uint32_t mt = (w[k] & 0x03030303u) * 0x01041040u;
-                sign |= (sg >> (28 - 4 * k)) & (0xFu << (4 * k));
-                mant |= (mt >> (24 - 8 * k)) & (0xFFu << (8 * k));
-            }
+        }
+        if (STORE) {
+            // Gathers by multiplication, in which no two partial products share
+            // a bit.  The sign bits of two words, the first word's shifted down
+            // by 4, land in order in the top byte of one product; the four 2-bit
+            // mantissas of a word land in order in the top byte of its product.
+            // Byte permutes then set the top bytes side by side.
+            const uint32_t s01 = (((w[0] & 0x80808080u) >> 4) | (w[1] & 0x80808080u)) * 0x00204081u;
+            const uint32_t s23 = (((w[2] & 0x80808080u) >> 4) | (w[3] & 0x80808080u)) * 0x00204081u;
+            sign = __byte_perm(s01, s23, 0x0073u);
+            uint32_t mt[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mt[k] = (w[k] & 0x03030303u) * 0x01041040u;
+            mant = __byte_perm(__byte_perm(mt[0], mt[1], 0x0073u), __byte_perm(mt[2], mt[3], 0x0073u), 0x5410u);
         }
         if (valid < 16) {
             if (valid < 8) {
@@ -509,6 +514,21 @@ __device__ __forceinline__ void rank_general(EMask<DT> m, uint4 v, uint32_t c, u
 // escapes are written then).
 template <int DT, typename Put>
 __device__ __forceinline__ void rank_step(EMask<DT> m, uint4 v, uint32_t &running, Put put, bool wanted = true) {
+    if constexpr (DT == SZ_FP8_E5M2) {
+        // one flag bit per escaped element: 4j for element j < 8, 4(j - 8) + 1 above
+        const uint32_t fl = uint32_t(m) | (uint32_t(m >> 32) << 1);
+        const uint32_t any = __ballot_sync(0xffffffffu, fl != 0u);
+        const uint32_t multi = __ballot_sync(0xffffffffu, (fl & (fl - 1u)) != 0u);
+        if (multi == 0u) {
+            // the escaped element's byte: byte (p >> 2) of words x, y (p even) or z, w (p odd)
+            const uint32_t p = __ffs(fl) - 1u;
+            const uint32_t odd = p & 1u;
+            const uint32_t e = (__byte_perm(odd ? v.z : v.x, odd ? v.w : v.y, p >> 2) >> 2) & 0x1Fu;
+            put(fl ? running + __popc(any & lanemask_lt()) : kNoRank, e);
+            running += __popc(any);
+            return;
+        }
+    }
     const uint32_t c = popc_mask(m);
     const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
     if (any == 0) return;
