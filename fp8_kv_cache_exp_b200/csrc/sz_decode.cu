@@ -4,7 +4,8 @@
 // bitwise identical to the originals; FAQ "How can I reduce KV cache transfer
 // time ...": decompression runs on the decode GPU.  The stored per-block
 // escape offsets make decode a pure gather with no dependency between blocks,
-// so one warp decodes one 4096-element block on its own, with no CTA barrier:
+// so one warp decodes one 4096-element block on its own, with no CTA barrier
+// on the way (one closes the kernel, before the last CTA resets the claims):
 //   - warps claim blocks one at a time from per-tensor counters (claiming the
 //     next block while decoding the current one), so they all finish within
 //     about one block of each other; a warp stays in one tensor while it has
@@ -20,8 +21,9 @@
 //     4-bit codes) select pre-spread exponent pairs from a 256-entry shared
 //     table, E5M2 codes select exponents from a 16-byte table in registers
 //     with prmt; escape ranks come from ballots (a fast path when no lane has
-//     two) and the escape bytes from a shuffle -- an E5M2 lane's single escape
-//     enters through its table's code-15 byte; the elements are reassembled
+//     two: in E5M2 it runs straight through, with one flag bit per escape and
+//     no per-lane counts) and the escape bytes from a shuffle -- an E5M2 lane's
+//     escape enters through its table's code-15 byte; the elements are reassembled
 //     with byte permutes and integer multiply-adds and written with 16-byte
 //     stores (512 contiguous bytes per warp instruction);
 //   - a raw block (header flag set and an offsets-table count equal to the

@@ -2,8 +2,8 @@
 //
 // SplitZip project page, Abstract: sign and mantissa bits are kept exactly,
 // frequent exponents get fixed 4-bit codes, rare exponents go to a sparse
-// escape stream.  Persistent CTAs of 8 independent warps (no CTA barrier on the
-// path).  Each warp takes chunks -- 1 to 8 consecutive 4096-element blocks of
+// escape stream.  Persistent CTAs of independent warps (8 per CTA for BF16, 12
+// for E5M2; no CTA barrier on the path).  Each warp takes chunks -- 1 to 8 consecutive 4096-element blocks of
 // one tensor, short chunks for small batches -- in launch order from an atomic
 // counter:
 //   1. the chunk's input arrives by 1-D bulk copies of 2 KB units into the
@@ -12,12 +12,13 @@
 //      shared load: exponent -> code through a 256-byte table whose entry
 //      address one prmt forms, sign|mantissa planes and 4-bit codes written
 //      with coalesced stores; escapes ranked by ballots (a fast path when no
-//      lane has two) and staged in element order in the warp's stage;
+//      lane has two; E5M2's takes one flag bit per escape and the exponent
+//      with one byte permute) and staged in element order in the warp's stage;
 //   3. the chunk's escape offset comes from a single-pass decoupled look-back
-//      over the chunks of its tensor (128 predecessors per step, resumable; a
-//      chunk whose predecessors have not yet published is finished once the
-//      warp has coded its next chunk; every wait is bounded: SZ_ERR_TIMEOUT
-//      instead of a hang);
+//      over the chunks of its tensor, on two levels (the chunk's own group of
+//      32 chunks, then whole groups, 32 per round); a chunk whose predecessors
+//      have not yet published is finished once the warp has coded its next
+//      chunk; every wait is bounded: SZ_ERR_TIMEOUT instead of a hang;
 //   4. the chunk's offsets-table entries and escapes are written contiguously
 //      (a chunk whose escapes overflow the stage re-codes its input and writes
 //      them directly); the tensor's last chunk writes the header, offsets[nb]
